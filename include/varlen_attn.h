@@ -1,0 +1,172 @@
+/*
+ * varlen_attn.h — C ABI of the packed variable-length attention forward
+ * library for NVIDIA B200 (sm_100a). Link: libvarlen_attn.so.
+ *
+ * The operation (pages cited by title and section):
+ *   Many ragged sequences are concatenated into one token stream; explicit
+ *   cumulative boundaries cu_seqlens say where each one starts, and each
+ *   sequence attends only to itself ("[feat] pack the GenRec training forward
+ *   through FlashAttention-2", summary and Test plan). Query heads share K/V
+ *   heads in groups (GQA: "fix(flex): avoid decoding kernel selection for
+ *   short GQA", Verification). An optional fp32 additive bias is either per
+ *   key or a dense per-pair grid read per sequence through strides (GiGL pull
+ *   request 858, Approach). For sequence i, query head h, local query row r
+ *   and local key c, with G = n_heads / n_kv_heads and kvh = h / G:
+ *
+ *     s = softmax_scale * <Q[cu_q[i]+r, h, :], K[cu_k[i]+c, kvh, :]>
+ *         + bias_per_key[cu_k[i]+c, h] + bias_pair[i*sb + h*sh + r*sq + c*sk]
+ *     visible(r, c) = !causal || c <= r + (Lk_i - Lq_i)     (bottom-right)
+ *     LSE[h, cu_q[i]+r] = ln sum_{visible c} exp(s)
+ *     out[cu_q[i]+r, h, :] = sum_{visible c} exp(s - LSE) * V[cu_k[i]+c, kvh, :]
+ *
+ *   A row that sees no key (or only -inf scores) gets out = 0, LSE = -inf.
+ *
+ * Conventions for every entry point:
+ *   - All array pointers are DEVICE pointers on the current CUDA device,
+ *     owned by the caller. The library never frees or keeps them.
+ *   - Sizes and scalars are host values. `stream` is a cudaStream_t passed as
+ *     void* (NULL = legacy default stream).
+ *   - Calls are asynchronous on `stream`: nothing synchronises, and outputs
+ *     are complete when the stream reaches the call.
+ *   - The library owns one grow-only device workspace per (device, stream)
+ *     for its work list; it is allocated on the first call that needs it (so
+ *     make a first call before timing or capturing). Calls on one stream are
+ *     ordered by the stream; calls on different streams use different
+ *     workspaces.
+ *   - Return value: VARLEN_ATTN_OK (0) or a positive varlen_attn_status.
+ *     Argument errors are detected on the host before anything is launched.
+ *     There is no fallback path: an unsupported case is an error.
+ *   - The contents of cu_seqlens are validated on the device (cu[0] = 0,
+ *     non-decreasing, cu[batch] <= total, each length <= its max_seqlen).
+ *     Invalid boundaries launch no attention work, leave out/lse unwritten and
+ *     raise VARLEN_ATTN_ERR_BAD_SEQLENS in the device error word, which
+ *     varlen_attn_get_device_error() reports.
+ */
+#ifndef VARLEN_ATTN_H_
+#define VARLEN_ATTN_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum varlen_attn_status {
+  VARLEN_ATTN_OK = 0,
+  VARLEN_ATTN_ERR_NULL_POINTER = 1,     /* a required pointer is NULL */
+  VARLEN_ATTN_ERR_BAD_SHAPE = 2,        /* batch/heads/totals/max lengths out of range,
+                                           or a zero-sized dimension (zero-dimension guard,
+                                           FDMA integration page, Key Implementation Points) */
+  VARLEN_ATTN_ERR_GQA_MISMATCH = 3,     /* n_heads is not a multiple of n_kv_heads */
+  VARLEN_ATTN_ERR_HEAD_DIM = 4,         /* head_dim not supported (bf16: 64 or 128;
+                                           fp32: 64 or 128) */
+  VARLEN_ATTN_ERR_MISALIGNED = 5,       /* q/k/v/out base not 16-byte aligned, or
+                                           lse/bias base not 4-byte aligned */
+  VARLEN_ATTN_ERR_BAD_BIAS = 6,         /* negative bias strides */
+  VARLEN_ATTN_ERR_CUDA = 7,             /* a CUDA runtime/driver call failed */
+  VARLEN_ATTN_ERR_DEVICE = 8,           /* current device is not sm_100 (B200 class) */
+  VARLEN_ATTN_ERR_BAD_SEQLENS = 9,      /* device-detected: cu_seqlens content invalid */
+  VARLEN_ATTN_ERR_DEVICE_TIMEOUT = 10,  /* device-detected: a bounded wait inside the
+                                           kernel expired; outputs are unspecified */
+  VARLEN_ATTN_ERR_TOO_LARGE = 11        /* sizes overflow the library's 32-bit indexing */
+} varlen_attn_status;
+
+/*
+ * Packed varlen attention forward, bf16 in / bf16 out, fp32 LSE.
+ * Runs on tensor cores (tcgen05, accumulators in tensor memory).
+ *
+ *   q        [total_q, n_heads, head_dim] bf16, contiguous, 16-byte aligned.
+ *   k, v     [total_k, n_kv_heads, head_dim] bf16, contiguous, 16-byte aligned.
+ *   cu_seqlens_q, cu_seqlens_k
+ *            [batch + 1] int32 device arrays; sequence i owns query rows
+ *            [cu_q[i], cu_q[i+1]) and key rows [cu_k[i], cu_k[i+1]).
+ *            Zero-length sequences are allowed.
+ *   batch    number of sequences B >= 1 (host value, so no device read is
+ *            needed to size the launch).
+ *   total_q, total_k
+ *            row counts of q and k/v (host values; the leading dimension of
+ *            the tensors). cu_q[B] <= total_q and cu_k[B] <= total_k.
+ *   max_seqlen_q, max_seqlen_k
+ *            upper bounds on the per-sequence lengths; they size the work list
+ *            and are checked on the device. Results do not depend on them.
+ *   n_heads, n_kv_heads
+ *            query heads Hq and K/V heads Hkv; Hq % Hkv == 0.
+ *   head_dim 64 or 128.
+ *   softmax_scale  multiplies <q, k> before the biases are added.
+ *   causal   0 or 1; 1 = bottom-right aligned mask c <= r + Lk - Lq.
+ *   bias_per_key   NULL, or [total_k, n_heads] fp32 contiguous.
+ *   bias_pair      NULL, or fp32 grid read at element offset
+ *                  i*bias_stride_b + h*bias_stride_h + r*bias_stride_q + c*bias_stride_k
+ *                  (strides in elements, >= 0; bias_stride_h = 0 shares one grid
+ *                  across heads). Only in-sequence entries (r < Lq_i, c < Lk_i) are
+ *                  read, so a grid sized [B, *, max_seqlen_q, max_seqlen_k] needs no
+ *                  zero padding (GiGL pull request 858, Approach, strided view).
+ *   out      [total_q, n_heads, head_dim] bf16 output, 16-byte aligned. Rows
+ *            outside every sequence (beyond cu_q[B]) are not written.
+ *   lse      NULL, or [n_heads, total_q] fp32 output: natural-log sum of exp of
+ *            the scaled, biased scores (-inf for a row that sees no key).
+ */
+int varlen_attn_fwd(const void* q, const void* k, const void* v,
+                    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                    int batch, int total_q, int total_k,
+                    int max_seqlen_q, int max_seqlen_k,
+                    int n_heads, int n_kv_heads, int head_dim,
+                    float softmax_scale, int causal,
+                    const float* bias_per_key,
+                    const float* bias_pair, int64_t bias_stride_b, int64_t bias_stride_h,
+                    int64_t bias_stride_q, int64_t bias_stride_k,
+                    void* out, float* lse, void* stream);
+
+/*
+ * Same operation with fp32 q/k/v/out (fp32 arithmetic on the CUDA cores).
+ * Same arguments and rules as varlen_attn_fwd, except that q, k, v and out
+ * are fp32 arrays of the same shapes. Meant for parity checks at fp32
+ * precision, where tensor-core TF32 rounding would be too coarse.
+ */
+int varlen_attn_fwd_f32(const float* q, const float* k, const float* v,
+                        const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                        int batch, int total_q, int total_k,
+                        int max_seqlen_q, int max_seqlen_k,
+                        int n_heads, int n_kv_heads, int head_dim,
+                        float softmax_scale, int causal,
+                        const float* bias_per_key,
+                        const float* bias_pair, int64_t bias_stride_b, int64_t bias_stride_h,
+                        int64_t bias_stride_q, int64_t bias_stride_k,
+                        float* out, float* lse, void* stream);
+
+/* Static description of a status code. Never NULL. */
+const char* varlen_attn_strerror(int status);
+
+/*
+ * Synchronises `stream`, then returns and clears the device error word of the
+ * current device (VARLEN_ATTN_OK if no kernel reported a problem). Returns
+ * VARLEN_ATTN_ERR_CUDA if the synchronisation itself fails.
+ */
+int varlen_attn_get_device_error(void* stream);
+
+/*
+ * Measurement hook. When both events are non-NULL, later calls from this host
+ * thread record `start_event` just before and `stop_event` just after the
+ * attention kernel's launch, on the call's stream (cudaEvent_t passed as
+ * void*). Pass NULL, NULL to stop. Does not change what is computed.
+ */
+int varlen_attn_set_profile_events(void* start_event, void* stop_event);
+
+/* Number of kernels one varlen_attn_fwd / varlen_attn_fwd_f32 call launches. */
+int varlen_attn_launches_per_call(int fp32_path);
+
+/*
+ * Detail of the last VARLEN_ATTN_ERR_CUDA raised on this host thread: the
+ * failing step and CUDA's message. Empty string if none. Never NULL; the
+ * buffer is owned by the library and overwritten by the next failure.
+ */
+const char* varlen_attn_last_error_detail(void);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int varlen_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VARLEN_ATTN_H_ */

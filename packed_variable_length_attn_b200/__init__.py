@@ -1,1 +1,203 @@
-"""packed_variable_length_attn_b200 (placeholder; the binding lands with the C ABI)."""
+"""Packed variable-length attention forward for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libvarlen_attn.so`` (declared in
+``include/varlen_attn.h``). This module only checks and marshals arguments:
+every step of the computation runs in the library's CUDA kernels. PyTorch
+provides device memory and the current stream. There is no fallback: if the
+library is missing or the device is not sm_100, calls raise.
+
+    out, lse = varlen_attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k,
+                               max_seqlen_q, max_seqlen_k, causal=True)
+
+``q`` is ``[total_q, n_heads, head_dim]``, ``k``/``v`` are
+``[total_k, n_kv_heads, head_dim]`` (bf16, or fp32 for the fp32 path),
+``cu_seqlens_*`` are int32 ``[batch + 1]`` on the same device. ``out`` has
+q's shape and dtype; ``lse`` is fp32 ``[n_heads, total_q]``.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Sequence, Tuple
+
+__all__ = ["varlen_attn_fwd", "library_path", "load_library", "VarlenAttnError",
+           "get_device_error", "set_profile_events", "launches_per_call", "exported_symbols"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libvarlen_attn.so")
+_lib = None
+
+# Status codes of include/varlen_attn.h
+OK = 0
+ERR_BAD_SEQLENS = 9
+ERR_DEVICE_TIMEOUT = 10
+
+
+class VarlenAttnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"varlen_attn error {status}: {message}")
+        self.status = status
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def exported_symbols() -> Tuple[str, ...]:
+    return ("varlen_attn_fwd", "varlen_attn_fwd_f32", "varlen_attn_strerror",
+            "varlen_attn_get_device_error", "varlen_attn_set_profile_events",
+            "varlen_attn_launches_per_call", "varlen_attn_version",
+            "varlen_attn_last_error_detail")
+
+
+def load_library():
+    """Load libvarlen_attn.so (built by build.py / __graft_entry__.build())."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"CUDA library not built: {_LIB_PATH} is missing "
+                          "(run packed_variable_length_attn_b200/build.py)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+    fwd_args = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, f32, i32, vp, vp,
+                i64, i64, i64, i64, vp, vp, vp]
+    lib.varlen_attn_fwd.argtypes = fwd_args
+    lib.varlen_attn_fwd.restype = i32
+    lib.varlen_attn_fwd_f32.argtypes = fwd_args
+    lib.varlen_attn_fwd_f32.restype = i32
+    lib.varlen_attn_strerror.argtypes = [i32]
+    lib.varlen_attn_strerror.restype = ctypes.c_char_p
+    lib.varlen_attn_get_device_error.argtypes = [vp]
+    lib.varlen_attn_get_device_error.restype = i32
+    lib.varlen_attn_set_profile_events.argtypes = [vp, vp]
+    lib.varlen_attn_set_profile_events.restype = i32
+    lib.varlen_attn_launches_per_call.argtypes = [i32]
+    lib.varlen_attn_launches_per_call.restype = i32
+    lib.varlen_attn_version.argtypes = []
+    lib.varlen_attn_version.restype = i32
+    lib.varlen_attn_last_error_detail.argtypes = []
+    lib.varlen_attn_last_error_detail.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def strerror(status: int) -> str:
+    return load_library().varlen_attn_strerror(int(status)).decode()
+
+
+def _check(status: int):
+    if status != OK:
+        msg = strerror(status)
+        if status == 7:
+            msg += " [" + load_library().varlen_attn_last_error_detail().decode() + "]"
+        raise VarlenAttnError(status, msg)
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def get_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error word."""
+    return int(load_library().varlen_attn_get_device_error(_stream_handle(stream)))
+
+
+def set_profile_events(start=None, stop=None):
+    """Record ``start``/``stop`` (torch.cuda.Event) around later attention-kernel
+    launches from this thread; ``set_profile_events()`` switches it off."""
+    lib = load_library()
+    if start is None or stop is None:
+        _check(lib.varlen_attn_set_profile_events(None, None))
+    else:
+        _check(lib.varlen_attn_set_profile_events(ctypes.c_void_p(start.cuda_event),
+                                                  ctypes.c_void_p(stop.cuda_event)))
+
+
+def launches_per_call(fp32: bool = False) -> int:
+    return int(load_library().varlen_attn_launches_per_call(1 if fp32 else 0))
+
+
+def _grid_strides(bias_pair, bias_pair_strides: Optional[Sequence[int]]):
+    if bias_pair_strides is not None:
+        return tuple(int(s) for s in bias_pair_strides)
+    if bias_pair.dim() != 4:
+        raise ValueError("bias_pair must be 4-D [batch, heads or 1, rows, cols] "
+                         "or come with explicit bias_pair_strides")
+    sb, sh, sr, sc = bias_pair.stride()
+    if bias_pair.shape[1] == 1:
+        sh = 0
+    return (sb, sh, sr, sc)
+
+
+def varlen_attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                    softmax_scale: Optional[float] = None, causal: bool = False,
+                    bias_per_key=None, bias_pair=None, bias_pair_strides=None,
+                    out=None, lse=None, return_lse: bool = True, stream=None):
+    """Packed variable-length attention forward through the C ABI.
+
+    bf16 q/k/v run the tensor-core kernel; fp32 q/k/v run the fp32 kernel.
+    ``bias_per_key``: fp32 ``[total_k, n_heads]``. ``bias_pair``: fp32 grid
+    read at ``i*sb + h*sh + r*sq + c*sk``; strides default to the tensor's own
+    (a 4-D ``[B, 1 or H, R, C]`` view, permuted views included; a size-1 head
+    axis broadcasts). Returns ``(out, lse)`` (``lse`` None if not requested).
+    """
+    import torch
+    lib = load_library()
+    if q.dim() != 3 or k.dim() != 3 or v.dim() != 3:
+        raise ValueError("q, k, v must be [tokens, heads, head_dim]")
+    if q.dtype not in (torch.bfloat16, torch.float32) or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must all be bf16 or all fp32")
+    tensors = [q, k, v, cu_seqlens_q, cu_seqlens_k]
+    for t in (bias_per_key, bias_pair, out, lse):
+        if t is not None:
+            tensors.append(t)
+    dev = q.device
+    if dev.type != "cuda" or any(t.device != dev for t in tensors):
+        raise ValueError("all tensors must be on the same CUDA device")
+    for name, t in (("q", q), ("k", k), ("v", v), ("cu_seqlens_q", cu_seqlens_q),
+                    ("cu_seqlens_k", cu_seqlens_k)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if cu_seqlens_q.dtype != torch.int32 or cu_seqlens_k.dtype != torch.int32:
+        raise ValueError("cu_seqlens must be int32")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have batch + 1 entries")
+    total_q, n_heads, head_dim = q.shape
+    total_k, n_kv_heads, dk = k.shape
+    if v.shape != k.shape or dk != head_dim:
+        raise ValueError("k and v must be [total_k, n_kv_heads, head_dim] like q's head_dim")
+    batch = cu_seqlens_q.numel() - 1
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(head_dim)
+    if bias_per_key is not None:
+        if bias_per_key.dtype != torch.float32 or not bias_per_key.is_contiguous() or \
+                tuple(bias_per_key.shape) != (total_k, n_heads):
+            raise ValueError("bias_per_key must be contiguous fp32 [total_k, n_heads]")
+    strides = (0, 0, 0, 0)
+    if bias_pair is not None:
+        if bias_pair.dtype != torch.float32:
+            raise ValueError("bias_pair must be fp32")
+        strides = _grid_strides(bias_pair, bias_pair_strides)
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous():
+        raise ValueError("out must be contiguous with q's shape and dtype")
+    if lse is None and return_lse:
+        lse = torch.empty((n_heads, total_q), dtype=torch.float32, device=dev)
+    elif lse is not None and (lse.shape != (n_heads, total_q) or lse.dtype != torch.float32
+                              or not lse.is_contiguous()):
+        raise ValueError("lse must be contiguous fp32 [n_heads, total_q]")
+    fn = lib.varlen_attn_fwd if q.dtype == torch.bfloat16 else lib.varlen_attn_fwd_f32
+    ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    with torch.cuda.device(dev):
+        status = fn(ptr(q), ptr(k), ptr(v), ptr(cu_seqlens_q), ptr(cu_seqlens_k), batch,
+                    total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), n_heads, n_kv_heads,
+                    head_dim, float(softmax_scale), 1 if causal else 0, ptr(bias_per_key),
+                    ptr(bias_pair), *strides, ptr(out), ptr(lse), _stream_handle(stream))
+    _check(status)
+    return out, lse

@@ -1,0 +1,593 @@
+// Packed variable-length attention forward for sm_100a (B200).
+//
+// Persistent, warp-specialised kernel; one CTA per SM, 12 warps in three
+// warpgroups:
+//   warps 0-3   softmax group 0: rows of slot 0 (thread = row = TMEM lane)
+//   warps 4-7   softmax group 1: rows of slot 1
+//   warp  8     MMA issue (one thread) + tensor-memory allocation
+//   warp  9     work fetch + TMA loads (one thread)
+//   warps 10-11 idle
+// The CTA launches with kLaunchRegs registers per thread; the third
+// warpgroup then gives registers up (setmaxnreg.dec to kWorkerRegs) and the
+// two softmax groups take them (setmaxnreg.inc to kSoftmaxRegs). The split
+// adds up exactly to the launch total, which the host checks against the
+// compiled kernel's register count before every first launch.
+//
+// A work item holds up to two 128-row query tiles ("slots") that stream the
+// same K/V tiles: two heads of one GQA group at one q-block, or two q-blocks
+// of one head. Per K/V tile j the tensor core computes S_s = Q_s K_j^T into
+// TMEM (fp32), the softmax group turns S_s into P_s (bf16, written back over
+// S_s in TMEM), and the tensor core accumulates O_s += P_s V_j in TMEM with P
+// read straight from tensor memory. The MMA order S0 S1 | PV0 S0' PV1 S1' |
+// ... lets one group's softmax run while the tensor core serves the other.
+//
+// Tensor memory (512 columns): S0/P0 [0,128), S1/P1 [128,256),
+// O0 [256, 256+D), O1 [256+D, 256+2D).
+//
+// Shared memory: Q0, Q1, then a ring of K/V tiles, each 128 rows x D bf16 in
+// 64-column, 128-byte-swizzled chunks as TMA writes them; per-key bias
+// staging; the work-item ring; mbarriers.
+//
+// Every mbarrier wait is bounded; on expiry the kernel records
+// kErrTimeout in the device error word, all roles leave their loops, the
+// loader waits (bounded) for its copies in flight, the MMA warp drains its
+// tensor-core work and frees tensor memory, and the CTA exits.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace va {
+
+constexpr int kAttnThreads = 384;
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 208;
+constexpr int kWorkerRegs = 88;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kWorkerRegs == kAttnThreads * kLaunchRegs,
+              "register split must add up to the launch allocation");
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+// A row's running max is only moved (and O rescaled) when the tile max
+// exceeds it by more than this many powers of two; P stays <= 2^8.
+constexpr float kRescaleThreshold = 8.0f;
+constexpr long long kWaitLimitCycles = 1ll << 33;    // ~4 s at 2 GHz
+constexpr long long kDrainLimitCycles = 1ll << 29;   // ~0.3 s
+
+template <int D>
+struct KCfg {
+  static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  static constexpr int kChunks = D / 64;
+  static constexpr int kChunkBytes = 128 * 128;      // 128 rows x 128 B
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kStages = D == 64 ? 8 : 4;    // K/V ring depth (tiles)
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = 2 * kTileBytes;
+  static constexpr int kBiasOff = kKVOff + kStages * kTileBytes;  // float [2 slot][2 buf][128]
+  static constexpr int kItemOff = kBiasOff + 2 * 2 * 128 * 4;
+  static constexpr int kBarOff = kItemOff + ((2 * (int)sizeof(Item) + 15) / 16) * 16;
+  // barriers: q_full[2] q_empty[2] s_full[2] p_full[2] o_full[2] o_empty[2]
+  //           item_full[2] item_empty[2] bias_full[2][2] drain kv_full[S] kv_empty[S]
+  static constexpr int kNumBars = 21 + 2 * kStages;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem slot, abort flag
+  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
+};
+
+struct Ctl {
+  volatile int* abort;
+  int* error;
+};
+
+__device__ __forceinline__ void raise_abort(const Ctl& c) {
+  *c.abort = 1;
+  atomicCAS(c.error, 0, kErrTimeout);
+}
+
+// Bounded wait for the phase of `bar` with the given parity.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const Ctl& c) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*c.abort) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      raise_abort(c);
+      return false;
+    }
+  }
+}
+
+// Bounded wait that ignores the abort flag (used to drain copies in flight).
+__device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!ptx::mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kDrainLimitCycles) return;
+  }
+}
+
+// UMMA shared-memory descriptors (sm_100 format, version 1).
+// K-major, 128-byte swizzle: rows 128 B apart, 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;                 // leading byte offset (unused for this layout)
+  d |= (uint64_t)(1024 >> 4) << 32;       // stride byte offset: next 8-row group
+  d |= (uint64_t)1 << 46;                 // descriptor version
+  d |= (uint64_t)2 << 61;                 // 128-byte swizzle
+  return d;
+}
+// MN-major, 128-byte swizzle: 64 MN-elements contiguous per 128-B row, K rows
+// 128 B apart, 8-row K groups 1024 B apart, 64-element MN chunks 16 KiB apart.
+__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(16384 >> 4) << 16;      // leading byte offset: next 64-wide MN chunk
+  d |= (uint64_t)(1024 >> 4) << 32;       // stride byte offset: next 8-row K group
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, M = 128.
+__host__ __device__ constexpr uint32_t idesc_bf16(int n, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+template <int D>
+struct Smem {
+  uint8_t* base;
+  __device__ uint8_t* q(int s) const { return base + KCfg<D>::kQOff + s * KCfg<D>::kTileBytes; }
+  __device__ uint8_t* kv(int st) const { return base + KCfg<D>::kKVOff + st * KCfg<D>::kTileBytes; }
+  __device__ float* bias(int s, int b) const {
+    return reinterpret_cast<float*>(base + KCfg<D>::kBiasOff) + (s * 2 + b) * 128;
+  }
+  __device__ Item* items() const { return reinterpret_cast<Item*>(base + KCfg<D>::kItemOff); }
+  __device__ uint64_t* bars() const { return reinterpret_cast<uint64_t*>(base + KCfg<D>::kBarOff); }
+  __device__ uint64_t* q_full(int s) const { return bars() + 0 + s; }
+  __device__ uint64_t* q_empty(int s) const { return bars() + 2 + s; }
+  __device__ uint64_t* s_full(int s) const { return bars() + 4 + s; }
+  __device__ uint64_t* p_full(int s) const { return bars() + 6 + s; }
+  __device__ uint64_t* o_full(int s) const { return bars() + 8 + s; }
+  __device__ uint64_t* o_empty(int s) const { return bars() + 10 + s; }
+  __device__ uint64_t* item_full(int k) const { return bars() + 12 + k; }
+  __device__ uint64_t* item_empty(int k) const { return bars() + 14 + k; }
+  __device__ uint64_t* bias_full(int s, int b) const { return bars() + 16 + s * 2 + b; }
+  __device__ uint64_t* drain() const { return bars() + 20; }
+  __device__ uint64_t* kv_full(int st) const { return bars() + 21 + st; }
+  __device__ uint64_t* kv_empty(int st) const { return bars() + 21 + KCfg<D>::kStages + st; }
+  __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + KCfg<D>::kMiscOff); }
+  __device__ int* abort_flag() const { return reinterpret_cast<int*>(base + KCfg<D>::kMiscOff + 4); }
+};
+
+__device__ __forceinline__ Item decode_item(int w, const AttnParams& p) {
+  Item it;
+  const int2 pr = p.ws.list[w / p.n_hg];
+  const int hg = w % p.n_hg;
+  const int i = pr.x, g = pr.y;
+  it.valid = 1;
+  it.seq = i;
+  const int q0 = p.cu_q[i], k0 = p.cu_k[i];
+  it.Lq = p.cu_q[i + 1] - q0;
+  it.Lk = p.cu_k[i + 1] - k0;
+  it.kv_row0 = k0;
+  it.kvh = p.pairing == kPairHeads ? hg / p.n_hp : hg / p.group;
+  fill_slots(it, g, hg, p.pairing, p.group, p.n_hp, p.causal);
+  it.q_row0[0] = q0 + it.q_loc0[0];
+  it.q_row0[1] = q0 + it.q_loc0[1];
+  return it;
+}
+
+// ------------------------------------------------------------------ loader
+template <int D>
+__device__ void load_role(const Smem<D>& sm, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                          const CUtensorMap* tm_v, const AttnParams& p, const Ctl& ctl) {
+  using C = KCfg<D>;
+  uint32_t kv_t = 0, q_uses[2] = {0, 0};
+  const int count = *reinterpret_cast<volatile int*>(p.ws.count);
+  for (int it = 0;; ++it) {
+    const int k = it & 1;
+    if (!wait_bar(sm.item_empty(k), ((it >> 1) & 1) ^ 1, ctl)) break;
+    const int w = atomicAdd(p.ws.counter, 1);
+    Item item;
+    if (w < count) {
+      item = decode_item(w, p);
+    } else {
+      item.valid = 0;
+    }
+    sm.items()[k] = item;
+    ptx::mbar_arrive(sm.item_full(k));
+    if (!item.valid) break;
+    bool ok = true;
+    for (int s = 0; s < 2 && ok; ++s) {
+      if (item.ntile[s] <= 0) continue;
+      if (!wait_bar(sm.q_empty(s), (q_uses[s] & 1) ^ 1, ctl)) { ok = false; break; }
+      ++q_uses[s];
+      ptx::mbar_arrive_expect_tx(sm.q_full(s), C::kTileBytes);
+      for (int c = 0; c < C::kChunks; ++c)
+        ptx::tma_load_3d(sm.q(s) + c * C::kChunkBytes, tm_q, sm.q_full(s), c * 64, item.head[s],
+                         item.q_row0[s]);
+    }
+    if (!ok) break;
+    const int n = max(item.ntile[0], item.ntile[1]);
+    for (int j = 0; j < n && ok; ++j) {
+      for (int kv = 0; kv < 2; ++kv) {
+        const int st = kv_t % C::kStages;
+        if (!wait_bar(sm.kv_empty(st), ((kv_t / C::kStages) & 1) ^ 1, ctl)) { ok = false; break; }
+        ++kv_t;
+        ptx::mbar_arrive_expect_tx(sm.kv_full(st), C::kTileBytes);
+        const CUtensorMap* tm = kv ? tm_v : tm_k;
+        for (int c = 0; c < C::kChunks; ++c)
+          ptx::tma_load_3d(sm.kv(st) + c * C::kChunkBytes, tm, sm.kv_full(st), c * 64, item.kvh,
+                           item.kv_row0 + j * BN);
+      }
+    }
+    if (!ok) break;
+  }
+  // Wait for every copy this thread started (immediate on the normal path).
+  for (int st = 0; st < C::kStages; ++st) {
+    if (kv_t > (uint32_t)st) {
+      const uint32_t uses = (kv_t - 1 - st) / C::kStages + 1;
+      drain_bar(sm.kv_full(st), (uses - 1) & 1);
+    }
+  }
+  for (int s = 0; s < 2; ++s)
+    if (q_uses[s] > 0) drain_bar(sm.q_full(s), (q_uses[s] - 1) & 1);
+}
+
+// ------------------------------------------------------------------ MMA issue
+template <int D>
+__device__ __forceinline__ void issue_s(const Smem<D>& sm, uint32_t tmem, int s, int kst) {
+  using C = KCfg<D>;
+  constexpr uint32_t idesc = idesc_bf16(BN, false);
+  const uint32_t qa = ptx::smem_u32(sm.q(s));
+  const uint32_t ka = ptx::smem_u32(sm.kv(kst));
+#pragma unroll
+  for (int k16 = 0; k16 < D / 16; ++k16) {
+    const uint32_t off = (k16 >> 2) * C::kChunkBytes + (k16 & 3) * 32;
+    ptx::mma_ss(tmem + s * 128, desc_kmajor_sw128(qa + off), desc_kmajor_sw128(ka + off), idesc,
+                k16 > 0);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(const Smem<D>& sm, uint32_t tmem, int s, int vst,
+                                         bool acc) {
+  constexpr uint32_t idesc = idesc_bf16(D, true);
+  const uint32_t va = ptx::smem_u32(sm.kv(vst));
+#pragma unroll
+  for (int k16 = 0; k16 < BN / 16; ++k16) {
+    ptx::mma_ts(tmem + 256 + s * D, tmem + s * 128 + k16 * 8,
+                desc_mnmajor_sw128(va + k16 * 16 * 128), idesc, (acc || k16 > 0) ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ void mma_role(const Smem<D>& sm, uint32_t tmem, const Ctl& ctl) {
+  using C = KCfg<D>;
+  uint32_t kv_t = 0, q_uses[2] = {0, 0}, p_uses[2] = {0, 0}, o_uses[2] = {0, 0};
+  for (int it = 0;; ++it) {
+    const int k = it & 1;
+    if (!wait_bar(sm.item_full(k), (it >> 1) & 1, ctl)) break;
+    const Item item = sm.items()[k];
+    ptx::mbar_arrive(sm.item_empty(k));
+    if (!item.valid) break;
+    const int nt[2] = {item.ntile[0], item.ntile[1]};
+    const int n = max(nt[0], nt[1]);
+    if (n == 0) continue;
+    bool ok = true;
+    for (int s = 0; s < 2 && ok; ++s) {
+      if (nt[s] <= 0) continue;
+      ok = wait_bar(sm.q_full(s), q_uses[s] & 1, ctl);
+      ++q_uses[s];
+    }
+    if (!ok) break;
+    // K_0 and the first scores
+    {
+      const int kst = kv_t % C::kStages;
+      if (!wait_bar(sm.kv_full(kst), (kv_t / C::kStages) & 1, ctl)) break;
+      ++kv_t;
+      ptx::tc_fence_after();
+      for (int s = 0; s < 2; ++s) {
+        if (nt[s] <= 0) continue;
+        issue_s<D>(sm, tmem, s, kst);
+        ptx::tc_commit(sm.s_full(s));
+        if (nt[s] == 1) ptx::tc_commit(sm.q_empty(s));
+      }
+      ptx::tc_commit(sm.kv_empty(kst));
+    }
+    for (int j = 0; j < n && ok; ++j) {
+      const int vst = kv_t % C::kStages;
+      if (!wait_bar(sm.kv_full(vst), (kv_t / C::kStages) & 1, ctl)) { ok = false; break; }
+      ++kv_t;
+      ptx::tc_fence_after();
+      int kst = -1;
+      for (int s = 0; s < 2; ++s) {
+        if (j < nt[s]) {
+          if (!wait_bar(sm.p_full(s), p_uses[s] & 1, ctl)) { ok = false; break; }
+          ++p_uses[s];
+          if (j == 0) {
+            if (!wait_bar(sm.o_empty(s), (o_uses[s] & 1) ^ 1, ctl)) { ok = false; break; }
+            ++o_uses[s];
+          }
+          ptx::tc_fence_after();
+          issue_pv<D>(sm, tmem, s, vst, j > 0);
+          if (j == nt[s] - 1) ptx::tc_commit(sm.o_full(s));
+        }
+        if (j + 1 < nt[s]) {
+          if (kst < 0) {
+            kst = kv_t % C::kStages;
+            if (!wait_bar(sm.kv_full(kst), (kv_t / C::kStages) & 1, ctl)) { ok = false; break; }
+            ++kv_t;
+            ptx::tc_fence_after();
+          }
+          issue_s<D>(sm, tmem, s, kst);
+          ptx::tc_commit(sm.s_full(s));
+          if (j + 2 == nt[s]) ptx::tc_commit(sm.q_empty(s));
+        }
+      }
+      if (!ok) break;
+      ptx::tc_commit(sm.kv_empty(vst));
+      if (kst >= 0) ptx::tc_commit(sm.kv_empty(kst));
+    }
+    if (!ok) break;
+  }
+  // Everything issued so far has completed once `drain` flips.
+  ptx::tc_commit(sm.drain());
+  drain_bar(sm.drain(), 0);
+}
+
+// Multiply this thread's O row (D fp32 columns of tensor memory) by fac.
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t t_o, float fac) {
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[32];
+    ptx::tmem_ld32(t_o + c * 32, o);
+    ptx::tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * fac);
+    ptx::tmem_st32(t_o + c * 32, o);
+  }
+  ptx::tmem_wait_st();
+}
+
+// ------------------------------------------------------------------ softmax
+template <int D, bool kBiasKey, bool kBiasPair>
+__device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams& p,
+                             const Ctl& ctl) {
+  const int warp = threadIdx.x >> 5;
+  const int wg = warp >> 2;                    // slot
+  const int r = threadIdx.x & 127;             // tile row = TMEM lane
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+  const uint32_t t_s = tmem + lane_base + wg * 128;
+  const uint32_t t_o = tmem + lane_base + 256 + wg * D;
+  const unsigned FULL = 0xffffffffu;
+  uint32_t s_uses = 0, o_uses = 0, b_uses = 0;
+  bool ok = true;
+
+  for (int it = 0; ok; ++it) {
+    const int k = it & 1;
+    ok = __all_sync(FULL, wait_bar(sm.item_full(k), (it >> 1) & 1, ctl));
+    if (!ok) break;
+    const Item item = sm.items()[k];
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(sm.item_empty(k));
+    if (!item.valid) break;
+    const int rows = item.rows[wg];
+    if (rows == 0) continue;
+    const int n = item.ntile[wg];
+    const int head = item.head[wg];
+    const int q_loc = item.q_loc0[wg] + r;
+    const bool row_ok = r < rows;
+    const int Lk = item.Lk;
+    const int limit = p.causal ? min(Lk, q_loc + (Lk - item.Lq) + 1) : Lk;
+    const float* brow = nullptr;
+    if (kBiasPair && row_ok)
+      brow = p.bias_pair + (long long)item.seq * p.sb + (long long)head * p.sh +
+             (long long)q_loc * p.sr;
+    float m_used = -INFINITY, l = 0.f;
+
+    for (int j = 0; j < n; ++j) {
+      const int kb = j * BN;
+      float* bk = nullptr;
+      if constexpr (kBiasKey) {
+        const int b = b_uses & 1;
+        bk = sm.bias(wg, b);
+        const int key = kb + r;
+        bk[r] = key < Lk ? p.bias_key[(long long)(item.kv_row0 + key) * p.n_heads + head] * kLog2e
+                         : 0.f;
+        ptx::mbar_arrive(sm.bias_full(wg, b));
+      }
+      ok = __all_sync(FULL, wait_bar(sm.s_full(wg), s_uses & 1, ctl));
+      if (!ok) break;
+      ++s_uses;
+      if constexpr (kBiasKey) {
+        ok = __all_sync(FULL, wait_bar(sm.bias_full(wg, b_uses & 1), (b_uses >> 1) & 1, ctl));
+        if (!ok) break;
+        ++b_uses;
+      }
+      ptx::tc_fence_after();
+      // One 128-register row buffer: raw scores -> log2-domain scores -> P.
+      uint32_t u[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        ptx::tmem_ld32(t_s + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c * 32]));
+      ptx::tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        float x;
+        if constexpr (kBiasKey)
+          x = fmaf(__uint_as_float(u[c]), p.scale_log2, bk[c]);
+        else
+          x = __uint_as_float(u[c]) * p.scale_log2;
+        u[c] = __float_as_uint(x);
+      }
+      if constexpr (kBiasPair) {
+        if (brow != nullptr) {
+#pragma unroll
+          for (int c = 0; c < 128; c += 4) {
+            const int key = kb + c;
+            if (p.pair_vec && key + 3 < Lk) {
+              const float4 b4 = __ldg(reinterpret_cast<const float4*>(brow + key));
+              u[c] = __float_as_uint(fmaf(b4.x, kLog2e, __uint_as_float(u[c])));
+              u[c + 1] = __float_as_uint(fmaf(b4.y, kLog2e, __uint_as_float(u[c + 1])));
+              u[c + 2] = __float_as_uint(fmaf(b4.z, kLog2e, __uint_as_float(u[c + 2])));
+              u[c + 3] = __float_as_uint(fmaf(b4.w, kLog2e, __uint_as_float(u[c + 3])));
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if (key + e < Lk)
+                  u[c + e] = __float_as_uint(
+                      fmaf(__ldg(brow + (long long)(key + e) * p.sc), kLog2e, __uint_as_float(u[c + e])));
+            }
+          }
+        }
+      }
+      if (__any_sync(FULL, kb + BN > limit)) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (kb + c >= limit) u[c] = __float_as_uint(-INFINITY);
+      }
+      float m_tile = __uint_as_float(u[0]);
+#pragma unroll
+      for (int c = 1; c < 128; ++c) m_tile = fmaxf(m_tile, __uint_as_float(u[c]));
+      const float m_new = fmaxf(m_used, m_tile);
+      const bool need = m_new > m_used + kRescaleThreshold;
+      float fac = 1.f;
+      if (need) {
+        fac = ptx::ex2(m_used - m_new);  // 0 when m_used is -inf
+        l *= fac;
+        m_used = m_new;
+      }
+      if (j > 0 && __any_sync(FULL, need)) rescale_o<D>(t_o, fac);
+      const float mb = m_used == -INFINITY ? 0.f : m_used;
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float p0 = ptx::ex2(__uint_as_float(u[2 * c]) - mb);
+        const float p1 = ptx::ex2(__uint_as_float(u[2 * c + 1]) - mb);
+        rs += p0 + p1;
+        u[c] = ptx::pack_bf16x2(p0, p1);  // u[c] is dead once u[2c], u[2c+1] are read
+      }
+      l += rs;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) ptx::tmem_st16(t_s + c * 16, &u[c * 16]);
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(sm.p_full(wg));
+    }
+    if (!ok) break;
+
+    // epilogue: O / l -> bf16, LSE
+    if (n > 0) {
+      ok = __all_sync(FULL, wait_bar(sm.o_full(wg), o_uses & 1, ctl));
+      if (!ok) break;
+      ++o_uses;
+      ptx::tc_fence_after();
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) +
+                          ((long long)(item.q_row0[wg] + r) * p.n_heads + head) * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      if (n > 0) {
+        ptx::tmem_ld32(t_o + c * 32, o);
+        ptx::tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = 0u;
+      }
+      if (row_ok) {
+        uint4 v[4];
+        uint32_t* vw = reinterpret_cast<uint32_t*>(v);
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          vw[e] = ptx::pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[e] = v[e];
+      }
+    }
+    if (n > 0) {
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(sm.o_empty(wg));
+    }
+    if (row_ok && p.lse != nullptr) {
+      const float lse = l > 0.f ? (m_used + __log2f(l)) * kLn2 : -INFINITY;
+      p.lse[(long long)head * p.total_q + item.q_row0[wg] + r] = lse;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ kernel
+template <int D, bool kBiasKey, bool kBiasPair>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem<D> sm;
+  {
+    const uint32_t a = ptx::smem_u32(smem_raw);
+    sm.base = smem_raw + ((1024 - (a & 1023)) & 1023);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(sm.q_full(s), 1);
+      ptx::mbar_init(sm.q_empty(s), 1);
+      ptx::mbar_init(sm.s_full(s), 1);
+      ptx::mbar_init(sm.p_full(s), 128);
+      ptx::mbar_init(sm.o_full(s), 1);
+      ptx::mbar_init(sm.o_empty(s), 128);
+      ptx::mbar_init(sm.item_full(s), 1);
+      ptx::mbar_init(sm.item_empty(s), 1 + 8);
+      ptx::mbar_init(sm.bias_full(s, 0), 128);
+      ptx::mbar_init(sm.bias_full(s, 1), 128);
+    }
+    ptx::mbar_init(sm.drain(), 1);
+    for (int st = 0; st < KCfg<D>::kStages; ++st) {
+      ptx::mbar_init(sm.kv_full(st), 1);
+      ptx::mbar_init(sm.kv_empty(st), 1);
+    }
+    *sm.abort_flag() = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    ptx::tmem_alloc(sm.tmem_slot(), 512);
+    ptx::tmem_relinquish();
+  }
+  if (warp == kLoadWarp && lane == 0) {
+    ptx::prefetch_tmap(&tm_q);
+    ptx::prefetch_tmap(&tm_k);
+    ptx::prefetch_tmap(&tm_v);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *sm.tmem_slot();
+  const Ctl ctl{sm.abort_flag(), p.error};
+
+  if (warp < 8) {
+    ptx::setmaxnreg_inc<kSoftmaxRegs>();
+    softmax_role<D, kBiasKey, kBiasPair>(sm, tmem, p, ctl);
+  } else {
+    ptx::setmaxnreg_dec<kWorkerRegs>();
+    if (warp == kMmaWarp) {
+      if (lane == 0) mma_role<D>(sm, tmem, ctl);
+      __syncwarp();
+    } else if (warp == kLoadWarp) {
+      if (lane == 0) load_role<D>(sm, &tm_q, &tm_k, &tm_v, p, ctl);
+      __syncwarp();
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace va

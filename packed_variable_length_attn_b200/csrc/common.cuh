@@ -1,0 +1,121 @@
+// Shared definitions of the packed varlen attention kernels: tile sizes,
+// launch parameters, the work item and its decoding from the work list.
+#pragma once
+#include <cstdint>
+
+namespace va {
+
+constexpr int BM = 128;  // query rows per slot tile (= TMEM lanes)
+constexpr int BN = 128;  // keys per K/V tile
+
+// Status codes (mirror varlen_attn_status in include/varlen_attn.h).
+constexpr int kErrBadSeqlens = 9;
+constexpr int kErrTimeout = 10;
+
+// How the two 128-row slots of a CTA work item are filled.
+//  kPairHeads:   two query heads of one K/V group at the same q-block (GQA:
+//                both slots read the same K/V tiles).
+//  kPairQBlocks: two consecutive q-blocks of one head (no GQA sharing).
+constexpr int kPairHeads = 0;
+constexpr int kPairQBlocks = 1;
+
+// Work list in the library workspace (device memory).
+struct Workspace {
+  int* counter;  // next work index (reset by the schedule kernel)
+  int* count;    // number of work items (0 = nothing to do / invalid input)
+  int2* list;    // sorted (sequence, group) pairs, `capacity` entries
+  int2* tmp;     // unsorted pairs, `capacity` entries
+  int capacity;
+};
+
+struct SchedParams {
+  const int* cu_q;
+  const int* cu_k;
+  int batch, total_q, total_k, max_q, max_k;
+  int causal;
+  int pairing;      // kPairHeads / kPairQBlocks; -1 = validate only
+  int n_hg;         // work items per (sequence, group) pair
+  Workspace ws;
+  int* error;       // device error word
+};
+
+struct AttnParams {
+  const int* cu_q;
+  const int* cu_k;
+  int total_q;
+  int n_heads, n_kv_heads, group;  // Hq, Hkv, G = Hq / Hkv
+  int pairing, n_hp, n_hg;
+  int causal;
+  float scale_log2;                // softmax_scale * log2(e)
+  const float* bias_key;           // [Tk, Hq] or null
+  const float* bias_pair;          // strided grid or null
+  long long sb, sh, sr, sc;
+  int pair_vec;                    // 1: 16-byte vector loads of the grid are legal
+  void* out;                       // bf16 [Tq, Hq, D]
+  float* lse;                      // [Hq, Tq] or null
+  Workspace ws;
+  int* error;
+};
+
+// One CTA work item: up to two 128-row query tiles (slots) that stream the
+// same K/V tiles of one K/V head.
+struct Item {
+  int valid;
+  int seq;
+  int kvh;
+  int kv_row0;   // cu_k[seq]
+  int Lq, Lk;
+  int q_row0[2]; // global first row of each slot
+  int q_loc0[2]; // first row of each slot, local to the sequence
+  int head[2];
+  int rows[2];   // valid rows in the slot (0 = slot unused)
+  int ntile[2];  // K/V tiles the slot needs (0 = no visible key)
+};
+
+__host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// K/V tiles a slot with local rows [q_loc0, q_loc0 + rows) must visit. With
+// the bottom-right causal mask the last row sees keys c < last + Lk - Lq + 1,
+// and fully masked tiles past that are skipped.
+__host__ __device__ __forceinline__ int slot_tiles(int q_loc0, int rows, int Lq, int Lk,
+                                                   int causal) {
+  if (rows <= 0 || Lk <= 0) return 0;
+  const int nk = ceil_div(Lk, BN);
+  if (!causal) return nk;
+  const int lim = q_loc0 + rows - 1 + (Lk - Lq) + 1;
+  if (lim <= 0) return 0;
+  const int n = ceil_div(lim, BN);
+  return n < nk ? n : nk;
+}
+
+// Number of (sequence, group) pairs sequence i contributes.
+__host__ __device__ __forceinline__ int seq_groups(int Lq, int pairing) {
+  const int nqb = ceil_div(Lq, BM);
+  return pairing == kPairHeads ? nqb : ceil_div(nqb, 2);
+}
+
+__device__ __forceinline__ void fill_slots(Item& it, int g, int hg, int pairing, int group,
+                                           int n_hp, int causal) {
+  for (int s = 0; s < 2; ++s) {
+    int active, head, q_loc0;
+    if (pairing == kPairHeads) {
+      const int hl = 2 * (hg % n_hp) + s;
+      active = hl < group;
+      head = it.kvh * group + hl;
+      q_loc0 = g * BM;
+    } else {
+      head = hg;
+      q_loc0 = (2 * g + s) * BM;
+      active = q_loc0 < it.Lq;
+    }
+    int rows = it.Lq - q_loc0;
+    rows = rows < BM ? rows : BM;
+    if (!active || rows < 0) rows = 0;
+    it.head[s] = head;
+    it.q_loc0[s] = q_loc0;
+    it.rows[s] = rows;
+    it.ntile[s] = slot_tiles(q_loc0, rows, it.Lq, it.Lk, causal);
+  }
+}
+
+}  // namespace va

@@ -1,0 +1,461 @@
+// Host side of the C ABI declared in include/varlen_attn.h: argument
+// validation, TMA descriptor encoding, the per-(device, stream) workspace,
+// and the launches of the schedule kernel and the attention kernel.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "../../include/varlen_attn.h"
+#include "attn_f32.cuh"
+#include "attn_sm100.cuh"
+#include "sched.cuh"
+
+namespace {
+
+using namespace va;
+
+__device__ int g_device_error = 0;
+
+constexpr int kVersion = 100;  // 0.1.0
+
+struct DeviceInfo {
+  bool init = false;
+  int sm_count = 0;
+  int cc_major = 0, cc_minor = 0;
+  int* error_word = nullptr;
+};
+
+std::mutex g_mu;
+std::map<int, DeviceInfo> g_dev;
+struct WsBuf {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+std::map<std::pair<int, void*>, WsBuf> g_ws;
+
+thread_local char t_detail[256] = "";
+
+// Records which step failed and CUDA's message; returns VARLEN_ATTN_ERR_CUDA.
+int cuda_fail(const char* step, cudaError_t e) {
+  snprintf(t_detail, sizeof t_detail, "%s: %s (%d)", step, cudaGetErrorString(e), (int)e);
+  return VARLEN_ATTN_ERR_CUDA;
+}
+
+thread_local cudaEvent_t t_ev_start = nullptr;
+thread_local cudaEvent_t t_ev_stop = nullptr;
+
+int device_info(DeviceInfo** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.init) {
+    if ((e = cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&di.cc_major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&di.cc_minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+      return cuda_fail("cudaDeviceGetAttribute", e);
+    if ((e = cudaGetSymbolAddress(reinterpret_cast<void**>(&di.error_word), g_device_error)) != cudaSuccess)
+      return cuda_fail("cudaGetSymbolAddress(error word)", e);
+    di.init = true;
+  }
+  if (di.cc_major != 10 || di.cc_minor != 0) return VARLEN_ATTN_ERR_DEVICE;
+  *out = &di;
+  return VARLEN_ATTN_OK;
+}
+
+// Grow-only workspace of `bytes` for (current device, stream).
+int workspace(void* stream, size_t bytes, void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+  std::lock_guard<std::mutex> lk(g_mu);
+  WsBuf& b = g_ws[std::make_pair(dev, stream)];
+  if (b.bytes < bytes) {
+    if (b.ptr != nullptr) {
+      // Earlier launches on this stream may still read the old buffer.
+      if ((e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream))) != cudaSuccess)
+        return cuda_fail("cudaStreamSynchronize(workspace growth)", e);
+      cudaFree(b.ptr);
+      b.ptr = nullptr;
+      b.bytes = 0;
+    }
+    size_t want = bytes < (1u << 16) ? (1u << 16) : bytes;
+    if ((e = cudaMalloc(&b.ptr, want)) != cudaSuccess) return cuda_fail("cudaMalloc(workspace)", e);
+    b.bytes = want;
+  }
+  *out = b.ptr;
+  return VARLEN_ATTN_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static cudaError_t err = cudaSuccess;
+  static int qres = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    err = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q);
+    qres = (int)q;
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  if (fn == nullptr)
+    snprintf(t_detail, sizeof t_detail, "cudaGetDriverEntryPointByVersion(cuTensorMapEncodeTiled): %s, query %d",
+             cudaGetErrorString(err), qres);
+  return fn;
+}
+
+// [rows, heads, D] bf16, box = 64 columns x 1 head x 128 rows, 128-byte swizzle.
+bool make_tmap(CUtensorMap* m, const void* base, int D, int heads, int rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)(rows > 0 ? rows : 1)};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) snprintf(t_detail, sizeof t_detail, "cuTensorMapEncodeTiled: CUresult %d", (int)r);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+struct Common {
+  int batch, total_q, total_k, max_q, max_k, Hq, Hkv, D, causal;
+  const int32_t *cu_q, *cu_k;
+  const float *bias_key, *bias_pair;
+  int64_t sb, sh, sr, sc;
+};
+
+int validate_common(const Common& a, const void* q, const void* k, const void* v, const void* out,
+                    const float* lse) {
+  if (!q || !k || !v || !out || !a.cu_q || !a.cu_k) return VARLEN_ATTN_ERR_NULL_POINTER;
+  if (a.batch <= 0 || a.Hq <= 0 || a.Hkv <= 0 || a.D <= 0 || a.total_q < 0 || a.total_k < 0 ||
+      a.max_q < 0 || a.max_k < 0)
+    return VARLEN_ATTN_ERR_BAD_SHAPE;
+  if (a.Hq % a.Hkv != 0) return VARLEN_ATTN_ERR_GQA_MISMATCH;
+  if (a.D != 64 && a.D != 128) return VARLEN_ATTN_ERR_HEAD_DIM;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+    return VARLEN_ATTN_ERR_MISALIGNED;
+  if ((lse && !aligned(lse, 4)) || (a.bias_key && !aligned(a.bias_key, 4)) ||
+      (a.bias_pair && !aligned(a.bias_pair, 4)) || !aligned(a.cu_q, 4) || !aligned(a.cu_k, 4))
+    return VARLEN_ATTN_ERR_MISALIGNED;
+  if (a.bias_pair && (a.sb < 0 || a.sh < 0 || a.sr < 0 || a.sc < 0)) return VARLEN_ATTN_ERR_BAD_BIAS;
+  // 32-bit indexing limits of the kernels.
+  if ((int64_t)a.total_q * a.Hq > INT32_MAX || (int64_t)a.total_k * a.Hkv > INT32_MAX ||
+      (int64_t)a.batch + 1 > INT32_MAX / 2)
+    return VARLEN_ATTN_ERR_TOO_LARGE;
+  return VARLEN_ATTN_OK;
+}
+
+template <typename K>
+int set_smem(K kernel, int bytes) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  return e == cudaSuccess ? VARLEN_ATTN_OK : cuda_fail("cudaFuncSetAttribute(smem)", e);
+}
+
+int check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? VARLEN_ATTN_OK : cuda_fail(what, e);
+}
+
+template <int D, bool BK, bool BP>
+int launch_attn(int grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                const AttnParams& prm, cudaStream_t st) {
+  auto kern = attn_fwd_sm100<D, BK, BP>;
+  static thread_local int configured_for = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_for != dev) {
+    // The in-kernel register split assumes exactly kLaunchRegs per thread at
+    // launch; with fewer, setmaxnreg.inc could never be satisfied.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return cuda_fail("cudaFuncGetAttributes", e);
+    if (fa.numRegs != kLaunchRegs) {
+      snprintf(t_detail, sizeof t_detail, "attn_fwd_sm100 compiled with %d registers, expected %d",
+               fa.numRegs, kLaunchRegs);
+      return VARLEN_ATTN_ERR_CUDA;
+    }
+    if (int rc = set_smem(kern, KCfg<D>::kSmemBytes)) return rc;
+    configured_for = dev;
+  }
+  kern<<<grid, kAttnThreads, KCfg<D>::kSmemBytes, st>>>(tq, tk, tv, prm);
+  return check_launch("launch attn_fwd_sm100");
+}
+
+int launch_schedule(const SchedParams& sp, cudaStream_t st) {
+  static thread_local int configured_for = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int smem = kSortCap * (int)sizeof(unsigned long long);
+  if (configured_for != dev) {
+    if (int rc = set_smem(schedule_kernel, smem)) return rc;
+    configured_for = dev;
+  }
+  schedule_kernel<<<1, kSchedThreads, smem, st>>>(sp);
+  return check_launch("launch schedule_kernel");
+}
+
+Workspace carve(void* base, int capacity) {
+  Workspace ws;
+  char* b = static_cast<char*>(base);
+  ws.counter = reinterpret_cast<int*>(b);
+  ws.count = reinterpret_cast<int*>(b + 4);
+  ws.list = reinterpret_cast<int2*>(b + 256);
+  ws.tmp = ws.list + capacity;
+  ws.capacity = capacity;
+  return ws;
+}
+
+}  // namespace
+
+extern "C" {
+
+int varlen_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                    const int32_t* cu_seqlens_k, int batch, int total_q, int total_k,
+                    int max_seqlen_q, int max_seqlen_k, int n_heads, int n_kv_heads, int head_dim,
+                    float softmax_scale, int causal, const float* bias_per_key,
+                    const float* bias_pair, int64_t bias_stride_b, int64_t bias_stride_h,
+                    int64_t bias_stride_q, int64_t bias_stride_k, void* out, float* lse,
+                    void* stream) {
+  Common a{batch, total_q, total_k, max_seqlen_q, max_seqlen_k, n_heads, n_kv_heads, head_dim,
+           causal ? 1 : 0, cu_seqlens_q, cu_seqlens_k, bias_per_key, bias_pair, bias_stride_b,
+           bias_stride_h, bias_stride_q, bias_stride_k};
+  int rc = validate_common(a, q, k, v, out, lse);
+  if (rc) return rc;
+  DeviceInfo* di = nullptr;
+  if ((rc = device_info(&di))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (total_q == 0 || max_seqlen_q == 0) return VARLEN_ATTN_OK;  // no query rows
+
+  const int G = n_heads / n_kv_heads;
+  const int pairing = G >= 2 ? kPairHeads : kPairQBlocks;
+  const int n_hp = (G + 1) / 2;
+  const int n_hg = pairing == kPairHeads ? n_kv_heads * n_hp : n_heads;
+  const int64_t groups_per_seq = seq_groups(max_seqlen_q, pairing);
+  const int64_t capacity = (int64_t)batch * groups_per_seq;
+  if (capacity * n_hg > INT32_MAX || capacity > (INT32_MAX / 16)) return VARLEN_ATTN_ERR_TOO_LARGE;
+
+  void* wsp = nullptr;
+  if ((rc = workspace(stream, 256 + 2 * (size_t)capacity * sizeof(int2), &wsp))) return rc;
+  Workspace ws = carve(wsp, (int)capacity);
+
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, head_dim, n_heads, total_q) ||
+      !make_tmap(&tk, k, head_dim, n_kv_heads, total_k) ||
+      !make_tmap(&tv, v, head_dim, n_kv_heads, total_k))
+    return VARLEN_ATTN_ERR_CUDA;
+
+  SchedParams sp;
+  sp.cu_q = cu_seqlens_q;
+  sp.cu_k = cu_seqlens_k;
+  sp.batch = batch;
+  sp.total_q = total_q;
+  sp.total_k = total_k;
+  sp.max_q = max_seqlen_q;
+  sp.max_k = max_seqlen_k;
+  sp.causal = a.causal;
+  sp.pairing = pairing;
+  sp.n_hg = n_hg;
+  sp.ws = ws;
+  sp.error = di->error_word;
+  if ((rc = launch_schedule(sp, st))) return rc;
+
+  AttnParams prm;
+  prm.cu_q = cu_seqlens_q;
+  prm.cu_k = cu_seqlens_k;
+  prm.total_q = total_q;
+  prm.n_heads = n_heads;
+  prm.n_kv_heads = n_kv_heads;
+  prm.group = G;
+  prm.pairing = pairing;
+  prm.n_hp = n_hp;
+  prm.n_hg = n_hg;
+  prm.causal = a.causal;
+  prm.scale_log2 = softmax_scale * 1.4426950408889634f;
+  prm.bias_key = bias_per_key;
+  prm.bias_pair = bias_pair;
+  prm.sb = bias_stride_b;
+  prm.sh = bias_stride_h;
+  prm.sr = bias_stride_q;
+  prm.sc = bias_stride_k;
+  prm.pair_vec = bias_pair && bias_stride_k == 1 && aligned(bias_pair, 16) &&
+                 bias_stride_b % 4 == 0 && bias_stride_h % 4 == 0 && bias_stride_q % 4 == 0;
+  prm.out = out;
+  prm.lse = lse;
+  prm.ws = ws;
+  prm.error = di->error_word;
+
+  int64_t items = capacity * n_hg;
+  const int grid = (int)(items < di->sm_count ? items : di->sm_count);
+  if (t_ev_start && t_ev_stop) {
+    cudaError_t e = cudaEventRecord(t_ev_start, st);
+    if (e != cudaSuccess) return cuda_fail("cudaEventRecord(start)", e);
+  }
+  const bool bk = bias_per_key != nullptr, bp = bias_pair != nullptr;
+  if (head_dim == 64) {
+    if (bk && bp) rc = launch_attn<64, true, true>(grid, tq, tk, tv, prm, st);
+    else if (bk) rc = launch_attn<64, true, false>(grid, tq, tk, tv, prm, st);
+    else if (bp) rc = launch_attn<64, false, true>(grid, tq, tk, tv, prm, st);
+    else rc = launch_attn<64, false, false>(grid, tq, tk, tv, prm, st);
+  } else {
+    if (bk && bp) rc = launch_attn<128, true, true>(grid, tq, tk, tv, prm, st);
+    else if (bk) rc = launch_attn<128, true, false>(grid, tq, tk, tv, prm, st);
+    else if (bp) rc = launch_attn<128, false, true>(grid, tq, tk, tv, prm, st);
+    else rc = launch_attn<128, false, false>(grid, tq, tk, tv, prm, st);
+  }
+  if (rc) return rc;
+  if (t_ev_start && t_ev_stop) {
+    cudaError_t e = cudaEventRecord(t_ev_stop, st);
+    if (e != cudaSuccess) return cuda_fail("cudaEventRecord(stop)", e);
+  }
+  return VARLEN_ATTN_OK;
+}
+
+int varlen_attn_fwd_f32(const float* q, const float* k, const float* v,
+                        const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch,
+                        int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
+                        int n_heads, int n_kv_heads, int head_dim, float softmax_scale,
+                        int causal, const float* bias_per_key, const float* bias_pair,
+                        int64_t bias_stride_b, int64_t bias_stride_h, int64_t bias_stride_q,
+                        int64_t bias_stride_k, float* out, float* lse, void* stream) {
+  Common a{batch, total_q, total_k, max_seqlen_q, max_seqlen_k, n_heads, n_kv_heads, head_dim,
+           causal ? 1 : 0, cu_seqlens_q, cu_seqlens_k, bias_per_key, bias_pair, bias_stride_b,
+           bias_stride_h, bias_stride_q, bias_stride_k};
+  int rc = validate_common(a, q, k, v, out, lse);
+  if (rc) return rc;
+  DeviceInfo* di = nullptr;
+  if ((rc = device_info(&di))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (total_q == 0 || max_seqlen_q == 0) return VARLEN_ATTN_OK;
+  const int64_t qblocks = ((int64_t)max_seqlen_q + kF32Rows - 1) / kF32Rows;
+  if ((int64_t)batch * qblocks > INT32_MAX || n_heads > 65535) return VARLEN_ATTN_ERR_TOO_LARGE;
+
+  void* wsp = nullptr;
+  if ((rc = workspace(stream, 256, &wsp))) return rc;
+  Workspace ws = carve(wsp, 0);
+  SchedParams sp;
+  std::memset(&sp, 0, sizeof sp);
+  sp.cu_q = cu_seqlens_q;
+  sp.cu_k = cu_seqlens_k;
+  sp.batch = batch;
+  sp.total_q = total_q;
+  sp.total_k = total_k;
+  sp.max_q = max_seqlen_q;
+  sp.max_k = max_seqlen_k;
+  sp.causal = a.causal;
+  sp.pairing = -1;  // validate only
+  sp.ws = ws;
+  sp.error = di->error_word;
+  if ((rc = launch_schedule(sp, st))) return rc;
+
+  F32Params prm;
+  prm.q = q;
+  prm.k = k;
+  prm.v = v;
+  prm.cu_q = cu_seqlens_q;
+  prm.cu_k = cu_seqlens_k;
+  prm.qblocks_max = (int)qblocks;
+  prm.total_q = total_q;
+  prm.n_heads = n_heads;
+  prm.group = n_heads / n_kv_heads;
+  prm.scale = softmax_scale;
+  prm.causal = a.causal;
+  prm.bias_key = bias_per_key;
+  prm.bias_pair = bias_pair;
+  prm.sb = bias_stride_b;
+  prm.sh = bias_stride_h;
+  prm.sr = bias_stride_q;
+  prm.sc = bias_stride_k;
+  prm.out = out;
+  prm.lse = lse;
+  prm.valid = ws.count;
+  dim3 grid((unsigned)(batch * qblocks), (unsigned)n_heads);
+  if (t_ev_start && t_ev_stop) {
+    cudaError_t e = cudaEventRecord(t_ev_start, st);
+    if (e != cudaSuccess) return cuda_fail("cudaEventRecord(start)", e);
+  }
+  if (head_dim == 64) {
+    static thread_local int cfg = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cfg != dev && (rc = set_smem(attn_fwd_f32<64>, F32Cfg<64>::kSmemBytes))) return rc;
+    cfg = dev;
+    attn_fwd_f32<64><<<grid, kF32Threads, F32Cfg<64>::kSmemBytes, st>>>(prm);
+  } else {
+    static thread_local int cfg = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cfg != dev && (rc = set_smem(attn_fwd_f32<128>, F32Cfg<128>::kSmemBytes))) return rc;
+    cfg = dev;
+    attn_fwd_f32<128><<<grid, kF32Threads, F32Cfg<128>::kSmemBytes, st>>>(prm);
+  }
+  if ((rc = check_launch("launch attn_fwd_f32"))) return rc;
+  if (t_ev_start && t_ev_stop) {
+    cudaError_t e = cudaEventRecord(t_ev_stop, st);
+    if (e != cudaSuccess) return cuda_fail("cudaEventRecord(stop)", e);
+  }
+  return VARLEN_ATTN_OK;
+}
+
+const char* varlen_attn_strerror(int status) {
+  switch (status) {
+    case VARLEN_ATTN_OK: return "ok";
+    case VARLEN_ATTN_ERR_NULL_POINTER: return "a required pointer is NULL";
+    case VARLEN_ATTN_ERR_BAD_SHAPE: return "batch, heads, totals or max lengths out of range";
+    case VARLEN_ATTN_ERR_GQA_MISMATCH: return "n_heads is not a multiple of n_kv_heads";
+    case VARLEN_ATTN_ERR_HEAD_DIM: return "head_dim must be 64 or 128";
+    case VARLEN_ATTN_ERR_MISALIGNED: return "q/k/v/out must be 16-byte aligned, lse/bias/cu_seqlens 4-byte aligned";
+    case VARLEN_ATTN_ERR_BAD_BIAS: return "bias strides must be non-negative";
+    case VARLEN_ATTN_ERR_CUDA: return "a CUDA call failed";
+    case VARLEN_ATTN_ERR_DEVICE: return "current device is not sm_100 (B200 class)";
+    case VARLEN_ATTN_ERR_BAD_SEQLENS: return "cu_seqlens content is invalid (device check)";
+    case VARLEN_ATTN_ERR_DEVICE_TIMEOUT: return "a bounded wait in the kernel expired";
+    case VARLEN_ATTN_ERR_TOO_LARGE: return "sizes exceed 32-bit indexing";
+    default: return "unknown status";
+  }
+}
+
+int varlen_attn_get_device_error(void* stream) {
+  DeviceInfo* di = nullptr;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail("cudaStreamSynchronize", e);
+  int v = 0;
+  if ((e = cudaMemcpy(&v, di->error_word, sizeof v, cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail("cudaMemcpy(error word)", e);
+  const int zero = 0;
+  if ((e = cudaMemcpy(di->error_word, &zero, sizeof zero, cudaMemcpyHostToDevice)) != cudaSuccess)
+    return cuda_fail("cudaMemcpy(error word reset)", e);
+  return v;
+}
+
+int varlen_attn_set_profile_events(void* start_event, void* stop_event) {
+  t_ev_start = static_cast<cudaEvent_t>(start_event);
+  t_ev_stop = static_cast<cudaEvent_t>(stop_event);
+  return VARLEN_ATTN_OK;
+}
+
+int varlen_attn_launches_per_call(int fp32_path) {
+  (void)fp32_path;
+  return 2;  // schedule (or validation) kernel + attention kernel
+}
+
+int varlen_attn_version(void) { return kVersion; }
+
+const char* varlen_attn_last_error_detail(void) { return t_detail; }
+
+}  // extern "C"

@@ -1,0 +1,94 @@
+"""CPU-side checks of the C-ABI library: it loads without a GPU, exports
+every entry point the header declares, and rejects bad arguments on the host
+before anything is launched. No compute call is made here."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import packed_variable_length_attn_b200 as va
+from packed_variable_length_attn_b200 import build as va_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    va_build.build()
+    return va.load_library()
+
+
+def _declared():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?\w+\s*\**\s*(varlen_attn_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert "varlen_attn_fwd" in names and "varlen_attn_fwd_f32" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(va.exported_symbols()) <= set(names) | set()
+    assert set(names) <= set(va.exported_symbols())
+
+
+def test_strerror_and_version(lib):
+    for code in range(0, 12):
+        assert va.strerror(code)
+    assert va.strerror(999) == "unknown status"
+    assert lib.varlen_attn_version() >= 100
+    assert va.launches_per_call() == 2
+
+
+def _call(lib, **kw):
+    a = dict(q=16, k=16, v=16, cu_q=16, cu_k=16, batch=1, total_q=8, total_k=8, max_q=8, max_k=8,
+             hq=2, hkv=2, d=64, scale=0.125, causal=1, bk=None, bp=None, sb=0, sh=0, sr=0, sc=0,
+             out=16, lse=16, stream=None)
+    a.update(kw)
+    p = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.varlen_attn_fwd(p(a["q"]), p(a["k"]), p(a["v"]), p(a["cu_q"]), p(a["cu_k"]),
+                               a["batch"], a["total_q"], a["total_k"], a["max_q"], a["max_k"],
+                               a["hq"], a["hkv"], a["d"], a["scale"], a["causal"], p(a["bk"]),
+                               p(a["bp"]), a["sb"], a["sh"], a["sr"], a["sc"], p(a["out"]),
+                               p(a["lse"]), a["stream"])
+
+
+def test_host_validation_codes(lib):
+    # the pointer values are never dereferenced: validation fails first
+    assert _call(lib, q=None) == 1
+    assert _call(lib, cu_k=None) == 1
+    assert _call(lib, batch=0) == 2
+    assert _call(lib, hq=0) == 2
+    assert _call(lib, total_q=-1) == 2
+    assert _call(lib, hq=3, hkv=2) == 3
+    assert _call(lib, d=96) == 4
+    assert _call(lib, d=256) == 4
+    assert _call(lib, q=24) == 5            # not 16-byte aligned
+    assert _call(lib, out=8) == 5
+    assert _call(lib, lse=18) == 5          # not 4-byte aligned
+    assert _call(lib, bp=16, sc=-1) == 6
+    assert _call(lib, total_q=1 << 30, hq=4, hkv=4) == 11
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU failure path")
+def test_no_device_is_an_error_not_a_fallback(lib):
+    # valid arguments on a machine without a GPU: a CUDA error code, no output
+    assert _call(lib) == 7
+    q = torch.zeros(8, 2, 64, dtype=torch.bfloat16)
+    cu = torch.tensor([0, 8], dtype=torch.int32)
+    with pytest.raises(ValueError):
+        va.varlen_attn_fwd(q, q, q, cu, cu, 8, 8)
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setattr(va, "_lib", None)
+    monkeypatch.setattr(va, "_LIB_PATH", "/nonexistent/libvarlen_attn.so")
+    with pytest.raises(ImportError):
+        va.load_library()
