@@ -1,0 +1,406 @@
+"""Benchmark: packed variable-length attention forward on B200.
+
+One step = one call of the C-ABI forward (schedule kernel + attention
+kernel) over one packed batch of the long causal GQA workload (16 sequences,
+lengths U[2048, 8192], 32 query / 8 K/V heads, head_dim 128, causal), inputs
+already resident in HBM. The batch is seeded and synthetic.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0). Under torchrun every rank runs its own batch
+(weak scaling: per-GPU work fixed, no data-path collective); the time is the
+max over ranks and the value the sum of all ranks' useful FLOPs over it.
+``--impl reference`` times the CPU oracle on bounded samples of the same
+workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "varlen attn fwd useful TFLOP/s & tokens/s on 1 B200; % of bf16 tensor peak"
+WORKLOAD = 5
+KERNEL_SOURCES = ["attn_sm100.cuh", "ptx.cuh", "common.cuh"]
+PROFILE_FILE = os.path.join(ROOT, "profiles", "attn_fwd_sm100_long_causal_gqa.md")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "packed_variable_length_attn_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _profiled_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source; else None."""
+    try:
+        txt = open(PROFILE_FILE).read()
+    except OSError:
+        return None
+    vals = {}
+    for line in txt.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_full_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in self.rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in self.rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4)
+                          if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _workload(args, seed=None):
+    from packed_variable_length_attn_b200 import workloads
+    w = workloads.make(WORKLOAD, seed=seed)
+    if args.sequences and args.sequences < w.batch:
+        n = args.sequences
+        tq, tk = int(w.cu_q[n]), int(w.cu_k[n])
+        w = workloads.Workload(f"{w.name}_first{n}", w.lengths_q[:n], w.lengths_k[:n],
+                               w.cu_q[:n + 1].clone(), w.cu_k[:n + 1].clone(), w.q[:tq].clone(),
+                               w.k[:tk].clone(), w.v[:tk].clone(), w.n_heads, w.n_kv_heads,
+                               w.head_dim, w.causal, w.softmax_scale, meta=dict(w.meta))
+    return w
+
+
+def run_reference(args, world, rank):
+    """The CPU oracle on bounded samples of the workload, on the host cores."""
+    if rank != 0:
+        return
+    w = _workload(args)
+    # size each step so that warm-up + timed steps take about args.ref_total_s
+    per_step = max(0.2, min(args.cpu_budget, args.ref_total_s / (args.steps + args.warmup)))
+    res = oracle_sample_rate(w, budget_s=per_step)
+    steps = args.steps
+    times = []
+    for _ in range(args.warmup):
+        oracle_sample_rate(w, budget_s=None, n_rows=res["n_rows"], seed=1)
+    for k in range(steps):
+        r = oracle_sample_rate(w, budget_s=None, n_rows=res["n_rows"], seed=2 + k)
+        times.append(r)
+    flops = sum(r["flops"] for r in times)
+    secs = sum(r["seconds"] for r in times)
+    value = flops / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": _config(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res["cores"],
+                         "kind": "oracle",
+                         "sample": f"{res['n_rows']} random (sequence, head, query row) outputs "
+                                   "of the workload per step, useful FLOPs of those rows"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def oracle_sample_rate(w, budget_s=None, n_rows=None, seed=0):
+    """Time oracle.rows on random output rows; returns flops, seconds, rows."""
+    import numpy as np
+    import oracle
+    cores = oracle.default_threads()
+    rng = np.random.default_rng(seed)
+
+    def pick(n):
+        seq = rng.integers(0, w.batch, n)
+        head = rng.integers(0, w.n_heads, n)
+        row = np.array([rng.integers(0, w.lengths_q[s]) for s in seq])
+        return seq, head, row
+
+    def flops_of(seq, row):
+        tot = 0
+        for s, r in zip(seq, row):
+            lq, lk = w.lengths_q[s], w.lengths_k[s]
+            nv = min(max(r + lk - lq + 1, 0), lk) if w.causal else lk
+            tot += 4 * w.head_dim * nv
+        return tot
+
+    def timed(n):
+        seq, head, row = pick(n)
+        t0 = time.perf_counter()
+        oracle.rows(w.q, w.k, w.v, w.cu_q, w.cu_k, w.n_heads, w.n_kv_heads, w.softmax_scale,
+                    w.causal, seq, head, row, threads=cores)
+        return flops_of(seq, row), time.perf_counter() - t0
+
+    if n_rows is None:
+        n = 4 * cores
+        f, s = timed(n)
+        while s < 0.5:
+            n *= 4
+            f, s = timed(n)
+        n_rows = max(1, int(n * budget_s / max(s, 1e-6)))
+    f, s = timed(n_rows)
+    return {"flops": f, "seconds": s, "n_rows": n_rows, "cores": cores}
+
+
+def _config(w):
+    from packed_variable_length_attn_b200 import metrics
+    pairs = metrics.useful_pairs(w.lengths_q, w.lengths_k, w.causal)
+    qkv_bytes = (w.q.numel() + w.k.numel() + w.v.numel()) * 2
+    return {"workload": w.name, "sequences": w.batch, "lengths": "uniform [2048, 8192]",
+            "lengths_drawn": list(w.lengths_q),
+            "total_tokens": w.total_q, "n_heads": w.n_heads, "n_kv_heads": w.n_kv_heads,
+            "head_dim": w.head_dim, "causal": w.causal, "bias": None,
+            "useful_pairs_per_head": pairs, "seed": w.meta.get("seed"),
+            "l2": f"inputs larger than L2 (Q+K+V {qkv_bytes / 1e9:.2f} GB > 126 MB); no flush"}
+
+
+def run_gpu(args, world, rank, local):
+    import torch
+    import torch.distributed as dist
+    import packed_variable_length_attn_b200 as va
+    from packed_variable_length_attn_b200 import metrics, workloads
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    seed = workloads.SEED_BASE + WORKLOAD + 1000 * rank
+    w = _workload(args, seed=seed)
+    flops = metrics.useful_flops(w.lengths_q, w.lengths_k, w.causal, w.n_heads, w.head_dim)
+    dev = torch.device("cuda", local)
+    q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
+    cu_q, cu_k = w.cu_q.to(dev), w.cu_k.to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.n_heads, w.total_q), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        va.varlen_attn_fwd(q, k, v, cu_q, cu_k, w.max_seqlen_q, w.max_seqlen_k,
+                           softmax_scale=w.softmax_scale, causal=True, out=out, lse=lse)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if va.get_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    # ---- timed region: K steps, device events, per-launch kernel events
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for a, b in kev:  # torch creates the CUDA events on first record
+        a.record(stream)
+        b.record(stream)
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)  # let the sampler start before the timed region
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        va.set_profile_events(*kev[i])
+        step()
+    va.set_profile_events()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    sampler.stop()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = t0.elapsed_time(t1)
+    kernel_ms = [a.elapsed_time(b) for a, b in kev]
+    if va.get_device_error() != 0:
+        raise RuntimeError("device error during the timed region")
+
+    # ---- end to end through host buffers (pinned), copies inside the region
+    hq, hk, hv = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
+    hcq, hck = cu_q.cpu().pin_memory(), cu_k.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    dq, dk_, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dcq, dck = torch.empty_like(cu_q), torch.empty_like(cu_k)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk_.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dcq.copy_(hcq, non_blocking=True)
+        dck.copy_(hck, non_blocking=True)
+        va.varlen_attn_fwd(dq, dk_, dv, dcq, dck, w.max_seqlen_q, w.max_seqlen_k,
+                           softmax_scale=w.softmax_scale, causal=True, out=out, lse=lse)
+        hout.copy_(out, non_blocking=True)
+        hlse.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e_steps = max(1, min(args.steps, args.e2e_steps))
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcq, hck))
+    d2h = hout.numel() * hout.element_size() + hlse.numel() * hlse.element_size()
+
+    # ---- reduce over ranks
+    stats = torch.tensor([elapsed_ms, e2e_ms, sum(kernel_ms) / len(kernel_ms)],
+                         dtype=torch.float64, device=dev)
+    tot = torch.tensor([float(flops), float(w.total_q)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
+        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
+    elapsed_ms, e2e_ms, kern_ms = stats.tolist()
+    all_flops, all_tokens = tot.tolist()
+
+    if rank == 0:
+        peaks, peak_src = _peaks()
+        ms_per_step = elapsed_ms / args.steps
+        value = all_flops / (ms_per_step * 1e-3) / 1e12
+        achieved = flops / (kern_ms * 1e-3) / 1e12  # this rank's kernel, per launch
+        peak = float(peaks["bf16_tflops"])
+        traffic = _profiled_traffic()
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 Q/K/V; lengths uniform [2048, 8192])",
+            "config": _config(w),
+            "tokens_per_s": all_tokens / (ms_per_step * 1e-3),
+            "pct_of_bf16_peak": 100.0 * value / (peak * world),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "frac_of_sustained": achieved / float(peaks["bf16_tflops_sustained"]),
+                         "kernel": "attn_fwd_sm100<128,false,false>",
+                         "kernel_ms_per_launch": kern_ms},
+            "e2e": {"value": all_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms, "steps": e_steps},
+            "gpu_launches": va.launches_per_call() * args.steps,
+            "clocks": sampler.summary(),
+        }
+        if not args.no_cpu_baseline:
+            r = oracle_sample_rate(w, budget_s=args.cpu_budget)
+            line["cpu_baseline"] = {
+                "value": r["flops"] / r["seconds"] / 1e12, "unit": "TFLOP/s",
+                "cores": r["cores"], "kind": "oracle",
+                "sample": f"{r['n_rows']} random (sequence, head, query row) outputs of the "
+                          f"workload, {r['seconds']:.1f} s, useful FLOPs of those rows"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-budget", type=float, default=12.0,
+                    help="seconds of oracle work for the CPU baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-total-s", type=float, default=150.0,
+                    help="--impl reference: seconds of oracle work over all steps")
+    ap.add_argument("--sequences", type=int, default=0,
+                    help="use only the first N sequences (small case for profiling)")
+    args = ap.parse_args()
+    world, rank, local = _dist()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    run_gpu(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

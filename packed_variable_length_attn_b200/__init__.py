@@ -114,6 +114,8 @@ def set_profile_events(start=None, stop=None):
     if start is None or stop is None:
         _check(lib.varlen_attn_set_profile_events(None, None))
     else:
+        if not start.cuda_event or not stop.cuda_event:
+            raise ValueError("record the events once first (torch creates them lazily)")
         _check(lib.varlen_attn_set_profile_events(ctypes.c_void_p(start.cuda_event),
                                                   ctypes.c_void_p(stop.cuda_event)))
 
