@@ -68,7 +68,9 @@ typedef enum varlen_attn_status {
   VARLEN_ATTN_ERR_BAD_SEQLENS = 9,      /* device-detected: cu_seqlens content invalid */
   VARLEN_ATTN_ERR_DEVICE_TIMEOUT = 10,  /* device-detected: a bounded wait inside the
                                            kernel expired; outputs are unspecified */
-  VARLEN_ATTN_ERR_TOO_LARGE = 11        /* sizes overflow the library's 32-bit indexing */
+  VARLEN_ATTN_ERR_TOO_LARGE = 11,       /* sizes overflow the library's 32-bit indexing */
+  VARLEN_ATTN_ERR_SCRATCH_LIMIT = 12    /* varlen_attn_fwd_noalloc: the work list does not
+                                           fit its fixed scratch */
 } varlen_attn_status;
 
 /*
@@ -133,6 +135,45 @@ int varlen_attn_fwd_f32(const float* q, const float* k, const float* v,
                         const float* bias_pair, int64_t bias_stride_b, int64_t bias_stride_h,
                         int64_t bias_stride_q, int64_t bias_stride_k,
                         float* out, float* lse, void* stream);
+
+/*
+ * varlen_attn_fwd without any device allocation by the library.
+ *
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot have a library allocate device memory on their behalf:
+ * runtimes that reserve the whole device pool up front and fail any outside
+ * cudaMalloc, request loops that must not stall (cudaMalloc/cudaFree can
+ * synchronise the device and take unbounded time), and hosts that give a
+ * plug-in a fixed memory budget.
+ *
+ * Same arguments, operation, outputs and rules as varlen_attn_fwd, except:
+ *   - The work list lives in a fixed array compiled into the library
+ *     (256 B + 2 x 16384 x 8 B, about 256 KiB) that every GPU loading the
+ *     library holds until the process exits. It calls no cudaMalloc,
+ *     cudaFree or other allocating routine; the caller still owns q/k/v,
+ *     the biases, out and lse.
+ *   - At most 16384 (sequence, q-block group) pairs: batch *
+ *     ceil(max_seqlen_q / 128) when n_heads / n_kv_heads >= 2, batch *
+ *     ceil(ceil(max_seqlen_q / 128) / 2) otherwise. Larger problems return
+ *     VARLEN_ATTN_ERR_SCRATCH_LIMIT before anything is launched.
+ *   - The first call on a device looks up that array's device address (with
+ *     the device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - Within a process, every call on a device shares that device's one
+ *     array, and each call overwrites what the previous call left there.
+ *     Calls that can run at the same time on one device (for example on two
+ *     streams) race on it; the caller must order them.
+ */
+int varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            int batch, int total_q, int total_k,
+                            int max_seqlen_q, int max_seqlen_k,
+                            int n_heads, int n_kv_heads, int head_dim,
+                            float softmax_scale, int causal,
+                            const float* bias_per_key,
+                            const float* bias_pair, int64_t bias_stride_b, int64_t bias_stride_h,
+                            int64_t bias_stride_q, int64_t bias_stride_k,
+                            void* out, float* lse, void* stream);
 
 /* Static description of a status code. Never NULL. */
 const char* varlen_attn_strerror(int status);

@@ -21,7 +21,7 @@ import math
 import os
 from typing import Optional, Sequence, Tuple
 
-__all__ = ["varlen_attn_fwd", "library_path", "load_library", "VarlenAttnError",
+__all__ = ["varlen_attn_fwd", "varlen_attn_fwd_noalloc", "library_path", "load_library", "VarlenAttnError",
            "get_device_error", "set_profile_events", "launches_per_call", "exported_symbols"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -48,7 +48,7 @@ def exported_symbols() -> Tuple[str, ...]:
     return ("varlen_attn_fwd", "varlen_attn_fwd_f32", "varlen_attn_strerror",
             "varlen_attn_get_device_error", "varlen_attn_set_profile_events",
             "varlen_attn_launches_per_call", "varlen_attn_version",
-            "varlen_attn_last_error_detail")
+            "varlen_attn_last_error_detail", "varlen_attn_fwd_noalloc")
 
 
 def load_library():
@@ -67,6 +67,8 @@ def load_library():
     lib.varlen_attn_fwd.restype = i32
     lib.varlen_attn_fwd_f32.argtypes = fwd_args
     lib.varlen_attn_fwd_f32.restype = i32
+    lib.varlen_attn_fwd_noalloc.argtypes = fwd_args
+    lib.varlen_attn_fwd_noalloc.restype = i32
     lib.varlen_attn_strerror.argtypes = [i32]
     lib.varlen_attn_strerror.restype = ctypes.c_char_p
     lib.varlen_attn_get_device_error.argtypes = [vp]
@@ -90,7 +92,7 @@ def strerror(status: int) -> str:
 def _check(status: int):
     if status != OK:
         msg = strerror(status)
-        if status == 7:
+        if status in (7, 12):
             msg += " [" + load_library().varlen_attn_last_error_detail().decode() + "]"
         raise VarlenAttnError(status, msg)
 
@@ -201,5 +203,47 @@ def varlen_attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_
                     total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), n_heads, n_kv_heads,
                     head_dim, float(softmax_scale), 1 if causal else 0, ptr(bias_per_key),
                     ptr(bias_pair), *strides, ptr(out), ptr(lse), _stream_handle(stream))
+    _check(status)
+    return out, lse
+
+
+def varlen_attn_fwd_noalloc(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
+                            max_seqlen_k: int, out, lse, softmax_scale: Optional[float] = None,
+                            causal: bool = False, bias_per_key=None, bias_pair=None,
+                            bias_pair_strides=None, stream=None):
+    """The same forward through ``varlen_attn_fwd_noalloc``: no device memory is
+    allocated, neither by the library (its work list sits in a fixed array of
+    the library, limited to 16384 (sequence, q-block group) pairs) nor here
+    (``out`` and ``lse`` must be given). For callers whose device memory is
+    managed elsewhere and must not be allocated behind their back. Calls that
+    can run concurrently on one device share that array and must be ordered.
+    bf16 only."""
+    import torch
+    lib = load_library()
+    if q.dtype != torch.bfloat16 or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("varlen_attn_fwd_noalloc takes bf16 q, k, v")
+    total_q, n_heads, head_dim = q.shape
+    total_k, n_kv_heads, _ = k.shape
+    if out is None or lse is None:
+        raise ValueError("out and lse must be provided (this path allocates nothing)")
+    if out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous():
+        raise ValueError("out must be contiguous with q's shape and dtype")
+    if lse.shape != (n_heads, total_q) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous fp32 [n_heads, total_q]")
+    for name, t in (("q", q), ("k", k), ("v", v), ("cu_seqlens_q", cu_seqlens_q),
+                    ("cu_seqlens_k", cu_seqlens_k)):
+        if not t.is_contiguous() or t.device != q.device:
+            raise ValueError(f"{name} must be contiguous and on q's device")
+    batch = cu_seqlens_q.numel() - 1
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(head_dim)
+    strides = (0, 0, 0, 0) if bias_pair is None else _grid_strides(bias_pair, bias_pair_strides)
+    ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    with torch.cuda.device(q.device):
+        status = lib.varlen_attn_fwd_noalloc(
+            ptr(q), ptr(k), ptr(v), ptr(cu_seqlens_q), ptr(cu_seqlens_k), batch, total_q,
+            total_k, int(max_seqlen_q), int(max_seqlen_k), n_heads, n_kv_heads, head_dim,
+            float(softmax_scale), 1 if causal else 0, ptr(bias_per_key), ptr(bias_pair),
+            *strides, ptr(out), ptr(lse), _stream_handle(stream))
     _check(status)
     return out, lse

@@ -17,6 +17,22 @@
 #include "attn_sm100.cuh"
 #include "sched.cuh"
 
+// ---------------------------------------------------------------------------
+// Fixed scratch for varlen_attn_fwd_noalloc.
+//
+// Some callers cannot let a library allocate device memory behind their
+// back: runtimes that reserve the whole device pool up front and fail any
+// outside cudaMalloc, serving loops that must not stall (cudaMalloc and
+// cudaFree can synchronise the device and take unbounded time), and hosts
+// that give a plug-in a fixed memory budget. For them the work list lives in
+// this array instead of the grow-only workspace. It is part of the library's
+// module: every GPU that loads the library holds it until the process exits.
+// All calls on one device share it, so calls that can run at the same time
+// on that device race on it.
+constexpr int kNoAllocMaxPairs = 16384;
+constexpr size_t kNoAllocScratchBytes = 256 + 2 * (size_t)kNoAllocMaxPairs * sizeof(int2);
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
 namespace {
 
 using namespace va;
@@ -219,6 +235,31 @@ Workspace carve(void* base, int capacity) {
   return ws;
 }
 
+// Device address of g_noalloc_scratch on the current device. In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+constexpr int kMaxDevices = 64;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+  if (dev < 0 || dev >= kMaxDevices) {
+    snprintf(t_detail, sizeof t_detail, "device ordinal %d beyond %d", dev, kMaxDevices);
+    return VARLEN_ATTN_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress(no-alloc scratch)", e);
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return VARLEN_ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -410,6 +451,106 @@ int varlen_attn_fwd_f32(const float* q, const float* k, const float* v,
   return VARLEN_ATTN_OK;
 }
 
+int varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch,
+                            int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
+                            int n_heads, int n_kv_heads, int head_dim, float softmax_scale,
+                            int causal, const float* bias_per_key, const float* bias_pair,
+                            int64_t bias_stride_b, int64_t bias_stride_h, int64_t bias_stride_q,
+                            int64_t bias_stride_k, void* out, float* lse, void* stream) {
+  Common a{batch, total_q, total_k, max_seqlen_q, max_seqlen_k, n_heads, n_kv_heads, head_dim,
+           causal ? 1 : 0, cu_seqlens_q, cu_seqlens_k, bias_per_key, bias_pair, bias_stride_b,
+           bias_stride_h, bias_stride_q, bias_stride_k};
+  int rc = validate_common(a, q, k, v, out, lse);
+  if (rc) return rc;
+  DeviceInfo* di = nullptr;
+  if ((rc = device_info(&di))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (total_q == 0 || max_seqlen_q == 0) return VARLEN_ATTN_OK;
+
+  const int G = n_heads / n_kv_heads;
+  const int pairing = G >= 2 ? kPairHeads : kPairQBlocks;
+  const int n_hp = (G + 1) / 2;
+  const int n_hg = pairing == kPairHeads ? n_kv_heads * n_hp : n_heads;
+  const int64_t capacity = (int64_t)batch * seq_groups(max_seqlen_q, pairing);
+  if (capacity > kNoAllocMaxPairs) {
+    snprintf(t_detail, sizeof t_detail,
+             "work list of %lld (sequence, q-block group) pairs exceeds the fixed scratch of %d",
+             (long long)capacity, kNoAllocMaxPairs);
+    return VARLEN_ATTN_ERR_SCRATCH_LIMIT;
+  }
+  if (capacity * n_hg > INT32_MAX) return VARLEN_ATTN_ERR_TOO_LARGE;
+
+  void* wsp = nullptr;
+  if ((rc = noalloc_scratch(&wsp))) return rc;
+  // The schedule kernel rewrites the counter, the count and every list entry
+  // it publishes before the attention kernel reads them, so no clearing of
+  // the previous call's contents is needed.
+  Workspace ws = carve(wsp, (int)capacity);
+
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, head_dim, n_heads, total_q) ||
+      !make_tmap(&tk, k, head_dim, n_kv_heads, total_k) ||
+      !make_tmap(&tv, v, head_dim, n_kv_heads, total_k))
+    return VARLEN_ATTN_ERR_CUDA;
+
+  SchedParams sp;
+  sp.cu_q = cu_seqlens_q;
+  sp.cu_k = cu_seqlens_k;
+  sp.batch = batch;
+  sp.total_q = total_q;
+  sp.total_k = total_k;
+  sp.max_q = max_seqlen_q;
+  sp.max_k = max_seqlen_k;
+  sp.causal = a.causal;
+  sp.pairing = pairing;
+  sp.n_hg = n_hg;
+  sp.ws = ws;
+  sp.error = di->error_word;
+  if ((rc = launch_schedule(sp, st))) return rc;
+
+  AttnParams prm;
+  prm.cu_q = cu_seqlens_q;
+  prm.cu_k = cu_seqlens_k;
+  prm.total_q = total_q;
+  prm.n_heads = n_heads;
+  prm.n_kv_heads = n_kv_heads;
+  prm.group = G;
+  prm.pairing = pairing;
+  prm.n_hp = n_hp;
+  prm.n_hg = n_hg;
+  prm.causal = a.causal;
+  prm.scale_log2 = softmax_scale * 1.4426950408889634f;
+  prm.bias_key = bias_per_key;
+  prm.bias_pair = bias_pair;
+  prm.sb = bias_stride_b;
+  prm.sh = bias_stride_h;
+  prm.sr = bias_stride_q;
+  prm.sc = bias_stride_k;
+  prm.pair_vec = bias_pair && bias_stride_k == 1 && aligned(bias_pair, 16) &&
+                 bias_stride_b % 4 == 0 && bias_stride_h % 4 == 0 && bias_stride_q % 4 == 0;
+  prm.out = out;
+  prm.lse = lse;
+  prm.ws = ws;
+  prm.error = di->error_word;
+
+  const int64_t items = capacity * n_hg;
+  const int grid = (int)(items < di->sm_count ? items : di->sm_count);
+  const bool bk = bias_per_key != nullptr, bp = bias_pair != nullptr;
+  if (head_dim == 64) {
+    if (bk && bp) rc = launch_attn<64, true, true>(grid, tq, tk, tv, prm, st);
+    else if (bk) rc = launch_attn<64, true, false>(grid, tq, tk, tv, prm, st);
+    else if (bp) rc = launch_attn<64, false, true>(grid, tq, tk, tv, prm, st);
+    else rc = launch_attn<64, false, false>(grid, tq, tk, tv, prm, st);
+  } else {
+    if (bk && bp) rc = launch_attn<128, true, true>(grid, tq, tk, tv, prm, st);
+    else if (bk) rc = launch_attn<128, true, false>(grid, tq, tk, tv, prm, st);
+    else if (bp) rc = launch_attn<128, false, true>(grid, tq, tk, tv, prm, st);
+    else rc = launch_attn<128, false, false>(grid, tq, tk, tv, prm, st);
+  }
+  return rc;
+}
+
 const char* varlen_attn_strerror(int status) {
   switch (status) {
     case VARLEN_ATTN_OK: return "ok";
@@ -424,6 +565,8 @@ const char* varlen_attn_strerror(int status) {
     case VARLEN_ATTN_ERR_BAD_SEQLENS: return "cu_seqlens content is invalid (device check)";
     case VARLEN_ATTN_ERR_DEVICE_TIMEOUT: return "a bounded wait in the kernel expired";
     case VARLEN_ATTN_ERR_TOO_LARGE: return "sizes exceed 32-bit indexing";
+    case VARLEN_ATTN_ERR_SCRATCH_LIMIT:
+      return "work list exceeds the fixed scratch of varlen_attn_fwd_noalloc";
     default: return "unknown status";
   }
 }
