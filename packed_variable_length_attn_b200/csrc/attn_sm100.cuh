@@ -4,8 +4,8 @@
 // warpgroups:
 //   warps 0-3   softmax group 0: rows of slot 0 (thread = row = TMEM lane)
 //   warps 4-7   softmax group 1: rows of slot 1
-//   warp  8     MMA issue (one thread) + tensor-memory allocation
-//   warp  9     work fetch + TMA loads (one thread)
+//   warp  8     MMA issue (one elected lane) + tensor-memory allocation
+//   warp  9     work fetch + TMA loads (one elected lane)
 //   warps 10-11 idle
 // The CTA launches with kLaunchRegs registers per thread; the third
 // warpgroup then gives registers up (setmaxnreg.dec to kWorkerRegs) and the
@@ -14,19 +14,22 @@
 // compiled kernel's register count before every first launch.
 //
 // A work item holds up to two 128-row query tiles ("slots") that stream the
-// same K/V tiles: two heads of one GQA group at one q-block, or two q-blocks
-// of one head. Per K/V tile j the tensor core computes S_s = Q_s K_j^T into
-// TMEM (fp32), the softmax group turns S_s into P_s (bf16, written back over
-// S_s in TMEM), and the tensor core accumulates O_s += P_s V_j in TMEM with P
-// read straight from tensor memory. The MMA order S0 S1 | PV0 S0' PV1 S1' |
-// ... lets one group's softmax run while the tensor core serves the other.
+// same 128-key K/V tiles: two heads of one GQA group at one q-block, or two
+// q-blocks of one head. Per K/V tile j the tensor core computes
+// S_s = Q_s K_j^T into tensor memory (fp32), the softmax group turns S_s into
+// P_s (bf16, written back over S_s), and the tensor core accumulates
+// O_s += P_s V_j with P read straight from tensor memory.
 //
 // Tensor memory (512 columns): S0/P0 [0,128), S1/P1 [128,256),
-// O0 [256, 256+D), O1 [256+D, 256+2D).
+// O0 [256, 256+D), O1 [256+D, 256+2D). The softmax publishes P in two halves
+// (keys 0-63, then 64-127), so the first half of P V runs on the tensor core
+// while the second half's exponentials are computed. MMA issue order:
+// S0(0) S1(0) | PV0a(j) PV0b(j) S0(j+1) PV1a(j) PV1b(j) S1(j+1) | ... : one
+// slot's softmax overlaps the other slot's MMAs.
 //
-// Shared memory: Q0, Q1, then a ring of K/V tiles, each 128 rows x D bf16 in
-// 64-column, 128-byte-swizzled chunks as TMA writes them; per-key bias
-// staging; the work-item ring; mbarriers.
+// Shared memory: Q0, Q1 (128 rows x D bf16, 64-column 128-byte-swizzled
+// chunks as TMA writes them), the K/V ring (128-row tiles, same layout),
+// per-key bias staging, the work-item ring, mbarriers.
 //
 // Every mbarrier wait is bounded; on expiry the kernel records
 // kErrTimeout in the device error word, all roles leave their loops, the
@@ -59,18 +62,21 @@ constexpr long long kDrainLimitCycles = 1ll << 29;   // ~0.3 s
 template <int D>
 struct KCfg {
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
-  static constexpr int kChunks = D / 64;
-  static constexpr int kChunkBytes = 128 * 128;      // 128 rows x 128 B
-  static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kStages = D == 64 ? 8 : 4;    // K/V ring depth (tiles)
+  static constexpr int kChunks = D / 64;                  // 64-column (128 B) chunks
+  static constexpr int kQChunk = BM * 128;                // 128 rows x 128 B
+  static constexpr int kKVChunk = BN * 128;               // 128 rows x 128 B
+  static constexpr int kQTile = kChunks * kQChunk;
+  static constexpr int kKVTile = kChunks * kKVChunk;
+  static constexpr int kStages = D == 64 ? 8 : 4;         // K/V ring depth (tiles)
   static constexpr int kQOff = 0;
-  static constexpr int kKVOff = 2 * kTileBytes;
-  static constexpr int kBiasOff = kKVOff + kStages * kTileBytes;  // float [2 slot][2 buf][128]
-  static constexpr int kItemOff = kBiasOff + 2 * 2 * 128 * 4;
+  static constexpr int kKVOff = 2 * kQTile;
+  static constexpr int kBiasOff = kKVOff + kStages * kKVTile;  // float [2 slot][2 buf][BN]
+  static constexpr int kItemOff = kBiasOff + 2 * 2 * BN * 4;
   static constexpr int kBarOff = kItemOff + ((2 * (int)sizeof(Item) + 15) / 16) * 16;
-  // barriers: q_full[2] q_empty[2] s_full[2] p_full[2] o_full[2] o_empty[2]
-  //           item_full[2] item_empty[2] bias_full[2][2] drain kv_full[S] kv_empty[S]
-  static constexpr int kNumBars = 21 + 2 * kStages;
+  // barriers: q_full[2] q_empty[2] s_full[2] p_full[2][2 halves] o_full[2]
+  //           o_empty[2] item_full[2] item_empty[2] bias_full[2][2] drain
+  //           kv_full[S] kv_empty[S]
+  static constexpr int kNumBars = 23 + 2 * kStages;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem slot, abort flag
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
 };
@@ -118,11 +124,11 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
   return d;
 }
 // MN-major, 128-byte swizzle: 64 MN-elements contiguous per 128-B row, K rows
-// 128 B apart, 8-row K groups 1024 B apart, 64-element MN chunks 16 KiB apart.
-__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t saddr) {
+// 128 B apart, 8-row K groups 1024 B apart, 64-element MN chunks `lbo` apart.
+__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t saddr, uint32_t lbo) {
   uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
-  d |= (uint64_t)(16384 >> 4) << 16;      // leading byte offset: next 64-wide MN chunk
-  d |= (uint64_t)(1024 >> 4) << 32;       // stride byte offset: next 8-row K group
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;  // leading byte offset: next 64-wide MN chunk
+  d |= (uint64_t)(1024 >> 4) << 32;             // stride byte offset: next 8-row K group
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)2 << 61;
   return d;
@@ -134,28 +140,33 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int n, bool b_mn_major) {
          ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
+// Tensor-memory columns.
+__device__ __forceinline__ uint32_t s_col(int s) { return (uint32_t)(s * 128); }
+template <int D>
+__device__ __forceinline__ uint32_t o_col(int s) { return (uint32_t)(256 + s * D); }
+
 template <int D>
 struct Smem {
   uint8_t* base;
-  __device__ uint8_t* q(int s) const { return base + KCfg<D>::kQOff + s * KCfg<D>::kTileBytes; }
-  __device__ uint8_t* kv(int st) const { return base + KCfg<D>::kKVOff + st * KCfg<D>::kTileBytes; }
+  __device__ uint8_t* q(int s) const { return base + KCfg<D>::kQOff + s * KCfg<D>::kQTile; }
+  __device__ uint8_t* kv(int st) const { return base + KCfg<D>::kKVOff + st * KCfg<D>::kKVTile; }
   __device__ float* bias(int s, int b) const {
-    return reinterpret_cast<float*>(base + KCfg<D>::kBiasOff) + (s * 2 + b) * 128;
+    return reinterpret_cast<float*>(base + KCfg<D>::kBiasOff) + (s * 2 + b) * BN;
   }
   __device__ Item* items() const { return reinterpret_cast<Item*>(base + KCfg<D>::kItemOff); }
   __device__ uint64_t* bars() const { return reinterpret_cast<uint64_t*>(base + KCfg<D>::kBarOff); }
   __device__ uint64_t* q_full(int s) const { return bars() + 0 + s; }
   __device__ uint64_t* q_empty(int s) const { return bars() + 2 + s; }
   __device__ uint64_t* s_full(int s) const { return bars() + 4 + s; }
-  __device__ uint64_t* p_full(int s) const { return bars() + 6 + s; }
-  __device__ uint64_t* o_full(int s) const { return bars() + 8 + s; }
-  __device__ uint64_t* o_empty(int s) const { return bars() + 10 + s; }
-  __device__ uint64_t* item_full(int k) const { return bars() + 12 + k; }
-  __device__ uint64_t* item_empty(int k) const { return bars() + 14 + k; }
-  __device__ uint64_t* bias_full(int s, int b) const { return bars() + 16 + s * 2 + b; }
-  __device__ uint64_t* drain() const { return bars() + 20; }
-  __device__ uint64_t* kv_full(int st) const { return bars() + 21 + st; }
-  __device__ uint64_t* kv_empty(int st) const { return bars() + 21 + KCfg<D>::kStages + st; }
+  __device__ uint64_t* p_full(int s, int h) const { return bars() + 6 + 2 * s + h; }
+  __device__ uint64_t* o_full(int s) const { return bars() + 10 + s; }
+  __device__ uint64_t* o_empty(int s) const { return bars() + 12 + s; }
+  __device__ uint64_t* item_full(int k) const { return bars() + 14 + k; }
+  __device__ uint64_t* item_empty(int k) const { return bars() + 16 + k; }
+  __device__ uint64_t* bias_full(int s, int b) const { return bars() + 18 + 2 * s + b; }
+  __device__ uint64_t* drain() const { return bars() + 22; }
+  __device__ uint64_t* kv_full(int st) const { return bars() + 23 + st; }
+  __device__ uint64_t* kv_empty(int st) const { return bars() + 23 + KCfg<D>::kStages + st; }
   __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + KCfg<D>::kMiscOff); }
   __device__ int* abort_flag() const { return reinterpret_cast<int*>(base + KCfg<D>::kMiscOff + 4); }
 };
@@ -179,52 +190,67 @@ __device__ __forceinline__ Item decode_item(int w, const AttnParams& p) {
 }
 
 // ------------------------------------------------------------------ loader
+// Runs on all 32 lanes of the load warp (uniform control flow); one elected
+// lane fetches work and issues the copies. Per item: Q of each active slot,
+// then K0, V0, K1, V1, ... (the MMA warp's consumption order).
 template <int D>
 __device__ void load_role(const Smem<D>& sm, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                           const CUtensorMap* tm_v, const AttnParams& p, const Ctl& ctl) {
   using C = KCfg<D>;
+  const unsigned FULL = 0xffffffffu;
   uint32_t kv_t = 0, q_uses[2] = {0, 0};
   const int count = *reinterpret_cast<volatile int*>(p.ws.count);
-  for (int it = 0;; ++it) {
-    const int k = it & 1;
-    if (!wait_bar(sm.item_empty(k), ((it >> 1) & 1) ^ 1, ctl)) break;
-    const int w = atomicAdd(p.ws.counter, 1);
-    Item item;
-    if (w < count) {
-      item = decode_item(w, p);
-    } else {
-      item.valid = 0;
+  bool ok = true;
+  auto load_kv = [&](const CUtensorMap* tm, int kvh, int row) {
+    const int st = kv_t % C::kStages;
+    if (!__all_sync(FULL, wait_bar(sm.kv_empty(st), ((kv_t / C::kStages) & 1) ^ 1, ctl))) {
+      ok = false;
+      return;
     }
-    sm.items()[k] = item;
-    ptx::mbar_arrive(sm.item_full(k));
+    ++kv_t;
+    if (ptx::elect_one()) {
+      ptx::mbar_arrive_expect_tx(sm.kv_full(st), C::kKVTile);
+      for (int c = 0; c < C::kChunks; ++c)
+        ptx::tma_load_3d(sm.kv(st) + c * C::kKVChunk, tm, sm.kv_full(st), c * 64, kvh, row);
+    }
+    __syncwarp();
+  };
+  for (int it = 0; ok; ++it) {
+    const int k = it & 1;
+    if (!__all_sync(FULL, wait_bar(sm.item_empty(k), ((it >> 1) & 1) ^ 1, ctl))) break;
+    if (ptx::elect_one()) {
+      const int w = atomicAdd(p.ws.counter, 1);
+      Item item;
+      if (w < count) {
+        item = decode_item(w, p);
+      } else {
+        item.valid = 0;
+      }
+      sm.items()[k] = item;
+      ptx::mbar_arrive(sm.item_full(k));
+    }
+    __syncwarp();
+    const Item item = sm.items()[k];
     if (!item.valid) break;
-    bool ok = true;
     for (int s = 0; s < 2 && ok; ++s) {
       if (item.ntile[s] <= 0) continue;
-      if (!wait_bar(sm.q_empty(s), (q_uses[s] & 1) ^ 1, ctl)) { ok = false; break; }
+      if (!__all_sync(FULL, wait_bar(sm.q_empty(s), (q_uses[s] & 1) ^ 1, ctl))) { ok = false; break; }
       ++q_uses[s];
-      ptx::mbar_arrive_expect_tx(sm.q_full(s), C::kTileBytes);
-      for (int c = 0; c < C::kChunks; ++c)
-        ptx::tma_load_3d(sm.q(s) + c * C::kChunkBytes, tm_q, sm.q_full(s), c * 64, item.head[s],
-                         item.q_row0[s]);
+      if (ptx::elect_one()) {
+        ptx::mbar_arrive_expect_tx(sm.q_full(s), C::kQTile);
+        for (int c = 0; c < C::kChunks; ++c)
+          ptx::tma_load_3d(sm.q(s) + c * C::kQChunk, tm_q, sm.q_full(s), c * 64, item.head[s],
+                           item.q_row0[s]);
+      }
+      __syncwarp();
     }
-    if (!ok) break;
     const int n = max(item.ntile[0], item.ntile[1]);
     for (int j = 0; j < n && ok; ++j) {
-      for (int kv = 0; kv < 2; ++kv) {
-        const int st = kv_t % C::kStages;
-        if (!wait_bar(sm.kv_empty(st), ((kv_t / C::kStages) & 1) ^ 1, ctl)) { ok = false; break; }
-        ++kv_t;
-        ptx::mbar_arrive_expect_tx(sm.kv_full(st), C::kTileBytes);
-        const CUtensorMap* tm = kv ? tm_v : tm_k;
-        for (int c = 0; c < C::kChunks; ++c)
-          ptx::tma_load_3d(sm.kv(st) + c * C::kChunkBytes, tm, sm.kv_full(st), c * 64, item.kvh,
-                           item.kv_row0 + j * BN);
-      }
+      load_kv(tm_k, item.kvh, item.kv_row0 + j * BN);
+      if (ok) load_kv(tm_v, item.kvh, item.kv_row0 + j * BN);
     }
-    if (!ok) break;
   }
-  // Wait for every copy this thread started (immediate on the normal path).
+  // Wait for every copy this warp started (immediate on the normal path).
   for (int st = 0; st < C::kStages; ++st) {
     if (kv_t > (uint32_t)st) {
       const uint32_t uses = (kv_t - 1 - st) / C::kStages + 1;
@@ -236,6 +262,7 @@ __device__ void load_role(const Smem<D>& sm, const CUtensorMap* tm_q, const CUte
 }
 
 // ------------------------------------------------------------------ MMA issue
+// S_s = Q_s K^T: M = 128, N = 128 keys, K = D in steps of 16.
 template <int D>
 __device__ __forceinline__ void issue_s(const Smem<D>& sm, uint32_t tmem, int s, int kst) {
   using C = KCfg<D>;
@@ -244,96 +271,127 @@ __device__ __forceinline__ void issue_s(const Smem<D>& sm, uint32_t tmem, int s,
   const uint32_t ka = ptx::smem_u32(sm.kv(kst));
 #pragma unroll
   for (int k16 = 0; k16 < D / 16; ++k16) {
-    const uint32_t off = (k16 >> 2) * C::kChunkBytes + (k16 & 3) * 32;
-    ptx::mma_ss(tmem + s * 128, desc_kmajor_sw128(qa + off), desc_kmajor_sw128(ka + off), idesc,
-                k16 > 0);
+    const uint32_t in = (k16 & 3) * 32;
+    ptx::mma_ss(tmem + s_col(s), desc_kmajor_sw128(qa + (k16 >> 2) * C::kQChunk + in),
+                desc_kmajor_sw128(ka + (k16 >> 2) * C::kKVChunk + in), idesc, k16 > 0);
   }
 }
 
+// O_s += P_s[keys 64h .. 64h+63] V[same keys]: M = 128, N = D, K = 64 in
+// steps of 16; P from tensor memory (2 keys per 32-bit column).
 template <int D>
-__device__ __forceinline__ void issue_pv(const Smem<D>& sm, uint32_t tmem, int s, int vst,
-                                         bool acc) {
+__device__ __forceinline__ void issue_pv_half(const Smem<D>& sm, uint32_t tmem, int s, int h,
+                                              int vst, bool acc) {
+  using C = KCfg<D>;
   constexpr uint32_t idesc = idesc_bf16(D, true);
   const uint32_t va = ptx::smem_u32(sm.kv(vst));
 #pragma unroll
-  for (int k16 = 0; k16 < BN / 16; ++k16) {
-    ptx::mma_ts(tmem + 256 + s * D, tmem + s * 128 + k16 * 8,
-                desc_mnmajor_sw128(va + k16 * 16 * 128), idesc, (acc || k16 > 0) ? 1u : 0u);
+  for (int k = 0; k < 4; ++k) {
+    const int k16 = 4 * h + k;
+    ptx::mma_ts(tmem + o_col<D>(s), tmem + s_col(s) + k16 * 8,
+                desc_mnmajor_sw128(va + k16 * 16 * 128, C::kKVChunk), idesc,
+                (acc || k16 > 0) ? 1u : 0u);
   }
 }
 
+// Runs on all 32 lanes of the MMA warp (uniform control flow); one elected
+// lane issues the tensor-core instructions and their commits.
 template <int D>
 __device__ void mma_role(const Smem<D>& sm, uint32_t tmem, const Ctl& ctl) {
   using C = KCfg<D>;
-  uint32_t kv_t = 0, q_uses[2] = {0, 0}, p_uses[2] = {0, 0}, o_uses[2] = {0, 0};
-  for (int it = 0;; ++it) {
+  const unsigned FULL = 0xffffffffu;
+  uint32_t kv_t = 0, q_uses[2] = {0, 0}, o_uses[2] = {0, 0};
+  uint32_t tc[2] = {0, 0};  // tiles issued per slot (phase of the P barriers)
+  auto wait = [&](uint64_t* bar, uint32_t parity) {
+    return __all_sync(FULL, wait_bar(bar, parity, ctl));
+  };
+  auto next_kv = [&](int& st) {
+    st = kv_t % C::kStages;
+    const bool r = wait(sm.kv_full(st), (kv_t / C::kStages) & 1);
+    ++kv_t;
+    return r;
+  };
+  bool ok = true;
+  for (int it = 0; ok; ++it) {
     const int k = it & 1;
-    if (!wait_bar(sm.item_full(k), (it >> 1) & 1, ctl)) break;
+    if (!wait(sm.item_full(k), (it >> 1) & 1)) break;
     const Item item = sm.items()[k];
-    ptx::mbar_arrive(sm.item_empty(k));
+    __syncwarp();
+    if (ptx::elect_one()) ptx::mbar_arrive(sm.item_empty(k));
     if (!item.valid) break;
     const int nt[2] = {item.ntile[0], item.ntile[1]};
     const int n = max(nt[0], nt[1]);
     if (n == 0) continue;
-    bool ok = true;
-    for (int s = 0; s < 2 && ok; ++s) {
-      if (nt[s] <= 0) continue;
-      ok = wait_bar(sm.q_full(s), q_uses[s] & 1, ctl);
-      ++q_uses[s];
-    }
-    if (!ok) break;
-    // K_0 and the first scores
-    {
-      const int kst = kv_t % C::kStages;
-      if (!wait_bar(sm.kv_full(kst), (kv_t / C::kStages) & 1, ctl)) break;
-      ++kv_t;
-      ptx::tc_fence_after();
-      for (int s = 0; s < 2; ++s) {
-        if (nt[s] <= 0) continue;
-        issue_s<D>(sm, tmem, s, kst);
-        ptx::tc_commit(sm.s_full(s));
-        if (nt[s] == 1) ptx::tc_commit(sm.q_empty(s));
+    for (int s = 0; s < 2 && ok; ++s)
+      if (nt[s] > 0) {
+        ok = wait(sm.q_full(s), q_uses[s] & 1);
+        ++q_uses[s];
       }
-      ptx::tc_commit(sm.kv_empty(kst));
+    if (!ok) break;
+    // K0 and the first scores
+    {
+      int kst;
+      if (!next_kv(kst)) break;
+      ptx::tc_fence_after();
+      if (ptx::elect_one()) {
+        for (int s = 0; s < 2; ++s) {
+          if (nt[s] <= 0) continue;
+          issue_s<D>(sm, tmem, s, kst);
+          ptx::tc_commit(sm.s_full(s));
+          if (nt[s] == 1) ptx::tc_commit(sm.q_empty(s));
+        }
+        ptx::tc_commit(sm.kv_empty(kst));
+      }
+      __syncwarp();
     }
     for (int j = 0; j < n && ok; ++j) {
-      const int vst = kv_t % C::kStages;
-      if (!wait_bar(sm.kv_full(vst), (kv_t / C::kStages) & 1, ctl)) { ok = false; break; }
-      ++kv_t;
-      ptx::tc_fence_after();
+      int vst;
+      if (!next_kv(vst)) { ok = false; break; }
       int kst = -1;
       for (int s = 0; s < 2; ++s) {
         if (j < nt[s]) {
-          if (!wait_bar(sm.p_full(s), p_uses[s] & 1, ctl)) { ok = false; break; }
-          ++p_uses[s];
+          const uint32_t ph = (tc[s] + j) & 1;
           if (j == 0) {
-            if (!wait_bar(sm.o_empty(s), (o_uses[s] & 1) ^ 1, ctl)) { ok = false; break; }
+            if (!wait(sm.o_empty(s), (o_uses[s] & 1) ^ 1)) { ok = false; break; }
             ++o_uses[s];
           }
-          ptx::tc_fence_after();
-          issue_pv<D>(sm, tmem, s, vst, j > 0);
-          if (j == nt[s] - 1) ptx::tc_commit(sm.o_full(s));
+          for (int h = 0; h < 2; ++h) {
+            if (!wait(sm.p_full(s, h), ph)) { ok = false; break; }
+            ptx::tc_fence_after();
+            if (ptx::elect_one()) {
+              issue_pv_half<D>(sm, tmem, s, h, vst, j > 0);
+              if (h == 1 && j == nt[s] - 1) ptx::tc_commit(sm.o_full(s));
+            }
+            __syncwarp();
+          }
+          if (!ok) break;
         }
         if (j + 1 < nt[s]) {
           if (kst < 0) {
-            kst = kv_t % C::kStages;
-            if (!wait_bar(sm.kv_full(kst), (kv_t / C::kStages) & 1, ctl)) { ok = false; break; }
-            ++kv_t;
+            if (!next_kv(kst)) { ok = false; break; }
             ptx::tc_fence_after();
           }
-          issue_s<D>(sm, tmem, s, kst);
-          ptx::tc_commit(sm.s_full(s));
-          if (j + 2 == nt[s]) ptx::tc_commit(sm.q_empty(s));
+          if (ptx::elect_one()) {
+            issue_s<D>(sm, tmem, s, kst);
+            ptx::tc_commit(sm.s_full(s));
+            if (j + 2 == nt[s]) ptx::tc_commit(sm.q_empty(s));
+          }
+          __syncwarp();
         }
       }
       if (!ok) break;
-      ptx::tc_commit(sm.kv_empty(vst));
-      if (kst >= 0) ptx::tc_commit(sm.kv_empty(kst));
+      if (ptx::elect_one()) {
+        ptx::tc_commit(sm.kv_empty(vst));
+        if (kst >= 0) ptx::tc_commit(sm.kv_empty(kst));
+      }
+      __syncwarp();
     }
-    if (!ok) break;
+    tc[0] += nt[0];
+    tc[1] += nt[1];
   }
   // Everything issued so far has completed once `drain` flips.
-  ptx::tc_commit(sm.drain());
+  if (ptx::elect_one()) ptx::tc_commit(sm.drain());
+  __syncwarp();
   drain_bar(sm.drain(), 0);
 }
 
@@ -360,10 +418,10 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
   const int wg = warp >> 2;                    // slot
   const int r = threadIdx.x & 127;             // tile row = TMEM lane
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-  const uint32_t t_s = tmem + lane_base + wg * 128;
-  const uint32_t t_o = tmem + lane_base + 256 + wg * D;
+  const uint32_t t_s = tmem + lane_base + s_col(wg);
+  const uint32_t t_o = tmem + lane_base + o_col<D>(wg);
   const unsigned FULL = 0xffffffffu;
-  uint32_t s_uses = 0, o_uses = 0, b_uses = 0;
+  uint32_t tc = 0, o_uses = 0;  // tiles processed (barrier phases), items with output
   bool ok = true;
 
   for (int it = 0; ok; ++it) {
@@ -390,43 +448,48 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
 
     for (int j = 0; j < n; ++j) {
       const int kb = j * BN;
+      const uint32_t g = tc + j;
+      const int b = g & 1;                   // bias staging buffer
+      const uint32_t ph = g & 1;             // phase of s_full / p_full for this tile
       float* bk = nullptr;
       if constexpr (kBiasKey) {
-        const int b = b_uses & 1;
         bk = sm.bias(wg, b);
         const int key = kb + r;
         bk[r] = key < Lk ? p.bias_key[(long long)(item.kv_row0 + key) * p.n_heads + head] * kLog2e
                          : 0.f;
         ptx::mbar_arrive(sm.bias_full(wg, b));
       }
-      ok = __all_sync(FULL, wait_bar(sm.s_full(wg), s_uses & 1, ctl));
+      ok = __all_sync(FULL, wait_bar(sm.s_full(wg), ph, ctl));
       if (!ok) break;
-      ++s_uses;
       if constexpr (kBiasKey) {
-        ok = __all_sync(FULL, wait_bar(sm.bias_full(wg, b_uses & 1), (b_uses >> 1) & 1, ctl));
+        ok = __all_sync(FULL, wait_bar(sm.bias_full(wg, b), (g >> 1) & 1, ctl));
         if (!ok) break;
-        ++b_uses;
       }
       ptx::tc_fence_after();
-      // One 128-register row buffer: raw scores -> log2-domain scores -> P.
-      uint32_t u[128];
+      // One 128-register row buffer: raw scores -> (log2-domain scores) -> P.
+      // Without a bias and with a positive scale the scores stay raw: the
+      // scale commutes with the row max and is folded into the exponent FMA.
+      uint32_t u[BN];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < BN / 32; ++c)
         ptx::tmem_ld32(t_s + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c * 32]));
       ptx::tmem_wait_ld();
+      const bool prescaled = kBiasKey || kBiasPair || !(p.scale_log2 > 0.f);
+      if (prescaled) {
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        float x;
-        if constexpr (kBiasKey)
-          x = fmaf(__uint_as_float(u[c]), p.scale_log2, bk[c]);
-        else
-          x = __uint_as_float(u[c]) * p.scale_log2;
-        u[c] = __float_as_uint(x);
+        for (int c = 0; c < BN; ++c) {
+          float x;
+          if constexpr (kBiasKey)
+            x = fmaf(__uint_as_float(u[c]), p.scale_log2, bk[c]);
+          else
+            x = __uint_as_float(u[c]) * p.scale_log2;
+          u[c] = __float_as_uint(x);
+        }
       }
       if constexpr (kBiasPair) {
         if (brow != nullptr) {
 #pragma unroll
-          for (int c = 0; c < 128; c += 4) {
+          for (int c = 0; c < BN; c += 4) {
             const int key = kb + c;
             if (p.pair_vec && key + 3 < Lk) {
               const float4 b4 = __ldg(reinterpret_cast<const float4*>(brow + key));
@@ -438,20 +501,31 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
 #pragma unroll
               for (int e = 0; e < 4; ++e)
                 if (key + e < Lk)
-                  u[c + e] = __float_as_uint(
-                      fmaf(__ldg(brow + (long long)(key + e) * p.sc), kLog2e, __uint_as_float(u[c + e])));
+                  u[c + e] = __float_as_uint(fmaf(__ldg(brow + (long long)(key + e) * p.sc),
+                                                  kLog2e, __uint_as_float(u[c + e])));
             }
           }
         }
       }
       if (__any_sync(FULL, kb + BN > limit)) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
+        for (int c = 0; c < BN; ++c)
           if (kb + c >= limit) u[c] = __float_as_uint(-INFINITY);
       }
-      float m_tile = __uint_as_float(u[0]);
+      // row max: a shallow tree of 3-input maxes (42 independent leaves)
+      float mx[43];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) m_tile = fmaxf(m_tile, __uint_as_float(u[c]));
+      for (int i = 0; i < 42; ++i)
+        mx[i] = ptx::fmax3(__uint_as_float(u[3 * i]), __uint_as_float(u[3 * i + 1]),
+                           __uint_as_float(u[3 * i + 2]));
+      mx[42] = fmaxf(__uint_as_float(u[126]), __uint_as_float(u[127]));
+#pragma unroll
+      for (int i = 0; i < 14; ++i) mx[i] = ptx::fmax3(mx[3 * i], mx[3 * i + 1], mx[3 * i + 2]);
+      mx[14] = mx[42];
+#pragma unroll
+      for (int i = 0; i < 5; ++i) mx[i] = ptx::fmax3(mx[3 * i], mx[3 * i + 1], mx[3 * i + 2]);
+      const float sfac = prescaled ? 1.f : p.scale_log2;
+      const float m_tile = ptx::fmax3(ptx::fmax3(mx[0], mx[1], mx[2]), mx[3], mx[4]) * sfac;
       const float m_new = fmaxf(m_used, m_tile);
       const bool need = m_new > m_used + kRescaleThreshold;
       float fac = 1.f;
@@ -460,24 +534,49 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
         l *= fac;
         m_used = m_new;
       }
+      // O_s already holds PV_s(j-1): S_s(j) was issued after it.
       if (j > 0 && __any_sync(FULL, need)) rescale_o<D>(t_o, fac);
       const float mb = m_used == -INFINITY ? 0.f : m_used;
-      float rs = 0.f;
+      // P = 2^(s * sfac - mb): one packed FMA per pair; three pairs in eight
+      // use the FMA-pipe polynomial, the rest the XU ex2. Each half of the
+      // keys is stored and published as soon as it is ready.
+      const uint64_t sf2 = ptx::f2(sfac, sfac), nm2 = ptx::f2(-mb, -mb);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = ptx::ex2(__uint_as_float(u[2 * c]) - mb);
-        const float p1 = ptx::ex2(__uint_as_float(u[2 * c + 1]) - mb);
-        rs += p0 + p1;
-        u[c] = ptx::pack_bf16x2(p0, p1);  // u[c] is dead once u[2c], u[2c+1] are read
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int cc = 0; cc < BN / 4; ++cc) {
+          const int c = h * (BN / 4) + cc;
+          const uint64_t x2 = ptx::ffma2(
+              ptx::f2(__uint_as_float(u[2 * c]), __uint_as_float(u[2 * c + 1])), sf2, nm2);
+          uint64_t p2;
+          if ((c & 7) == 2 || (c & 7) == 5 || (c & 7) == 7) {
+            p2 = ptx::exp2_poly2(x2);
+          } else {
+            float x0, x1;
+            ptx::f2_split(x2, x0, x1);
+            p2 = ptx::f2(ptx::ex2(x0), ptx::ex2(x1));
+          }
+          acc[c & 3] = ptx::fadd2(acc[c & 3], p2);
+          float p0, p1;
+          ptx::f2_split(p2, p0, p1);
+          u[c] = ptx::pack_bf16x2(p0, p1);  // u[c] is dead once u[2c], u[2c+1] are read
+        }
+        ptx::tmem_st16(t_s + h * 32, &u[h * 32]);
+        ptx::tmem_st16(t_s + h * 32 + 16, &u[h * 32 + 16]);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(sm.p_full(wg, h));
       }
-      l += rs;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) ptx::tmem_st16(t_s + c * 16, &u[c * 16]);
-      ptx::tmem_wait_st();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(sm.p_full(wg));
+      {
+        const uint64_t s01 = ptx::fadd2(ptx::fadd2(acc[0], acc[1]), ptx::fadd2(acc[2], acc[3]));
+        float r0, r1;
+        ptx::f2_split(s01, r0, r1);
+        l += r0 + r1;
+      }
     }
     if (!ok) break;
+    tc += n;
 
     // epilogue: O / l -> bf16, LSE
     if (n > 0) {
@@ -538,13 +637,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ptx::mbar_init(sm.q_full(s), 1);
       ptx::mbar_init(sm.q_empty(s), 1);
       ptx::mbar_init(sm.s_full(s), 1);
-      ptx::mbar_init(sm.p_full(s), 128);
+      for (int b = 0; b < 2; ++b) {
+        ptx::mbar_init(sm.p_full(s, b), 128);
+        ptx::mbar_init(sm.bias_full(s, b), 128);
+      }
       ptx::mbar_init(sm.o_full(s), 1);
       ptx::mbar_init(sm.o_empty(s), 128);
       ptx::mbar_init(sm.item_full(s), 1);
       ptx::mbar_init(sm.item_empty(s), 1 + 8);
-      ptx::mbar_init(sm.bias_full(s, 0), 128);
-      ptx::mbar_init(sm.bias_full(s, 1), 128);
     }
     ptx::mbar_init(sm.drain(), 1);
     for (int st = 0; st < KCfg<D>::kStages; ++st) {
@@ -575,11 +675,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else {
     ptx::setmaxnreg_dec<kWorkerRegs>();
     if (warp == kMmaWarp) {
-      if (lane == 0) mma_role<D>(sm, tmem, ctl);
-      __syncwarp();
+      mma_role<D>(sm, tmem, ctl);
     } else if (warp == kLoadWarp) {
-      if (lane == 0) load_role<D>(sm, &tm_q, &tm_k, &tm_v, p, ctl);
-      __syncwarp();
+      load_role<D>(sm, &tm_q, &tm_k, &tm_v, p, ctl);
     }
   }
   ptx::tc_fence_before();

@@ -130,13 +130,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [rows, heads, D] bf16, box = 64 columns x 1 head x 128 rows, 128-byte swizzle.
-bool make_tmap(CUtensorMap* m, const void* base, int D, int heads, int rows) {
+// [rows, heads, D] bf16, box = 64 columns x 1 head x box_rows rows, 128-byte swizzle.
+bool make_tmap(CUtensorMap* m, const void* base, int D, int heads, int rows, int box_rows) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)(rows > 0 ? rows : 1)};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
-  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -294,9 +294,9 @@ int varlen_attn_fwd(const void* q, const void* k, const void* v, const int32_t* 
   Workspace ws = carve(wsp, (int)capacity);
 
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, head_dim, n_heads, total_q) ||
-      !make_tmap(&tk, k, head_dim, n_kv_heads, total_k) ||
-      !make_tmap(&tv, v, head_dim, n_kv_heads, total_k))
+  if (!make_tmap(&tq, q, head_dim, n_heads, total_q, BM) ||
+      !make_tmap(&tk, k, head_dim, n_kv_heads, total_k, BN) ||
+      !make_tmap(&tv, v, head_dim, n_kv_heads, total_k, BN))
     return VARLEN_ATTN_ERR_CUDA;
 
   SchedParams sp;
@@ -489,9 +489,9 @@ int varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   Workspace ws = carve(wsp, (int)capacity);
 
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, head_dim, n_heads, total_q) ||
-      !make_tmap(&tk, k, head_dim, n_kv_heads, total_k) ||
-      !make_tmap(&tv, v, head_dim, n_kv_heads, total_k))
+  if (!make_tmap(&tq, q, head_dim, n_heads, total_q, BM) ||
+      !make_tmap(&tk, k, head_dim, n_kv_heads, total_k, BN) ||
+      !make_tmap(&tv, v, head_dim, n_kv_heads, total_k, BN))
     return VARLEN_ATTN_ERR_CUDA;
 
   SchedParams sp;
