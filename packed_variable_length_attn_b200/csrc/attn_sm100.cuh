@@ -45,8 +45,8 @@ namespace va {
 
 constexpr int kAttnThreads = 384;
 constexpr int kLaunchRegs = 168;
-constexpr int kSoftmaxRegs = 208;
-constexpr int kWorkerRegs = 88;
+constexpr int kSoftmaxRegs = 200;
+constexpr int kWorkerRegs = 104;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kWorkerRegs == kAttnThreads * kLaunchRegs,
               "register split must add up to the launch allocation");
 constexpr int kMmaWarp = 8;
@@ -232,17 +232,19 @@ __device__ void load_role(const Smem<D>& sm, const CUtensorMap* tm_q, const CUte
     __syncwarp();
     const Item item = sm.items()[k];
     if (!item.valid) break;
-    for (int s = 0; s < 2 && ok; ++s) {
-      if (item.ntile[s] <= 0) continue;
-      if (!__all_sync(FULL, wait_bar(sm.q_empty(s), (q_uses[s] & 1) ^ 1, ctl))) { ok = false; break; }
-      ++q_uses[s];
-      if (ptx::elect_one()) {
-        ptx::mbar_arrive_expect_tx(sm.q_full(s), C::kQTile);
-        for (int c = 0; c < C::kChunks; ++c)
-          ptx::tma_load_3d(sm.q(s) + c * C::kQChunk, tm_q, sm.q_full(s), c * 64, item.head[s],
-                           item.q_row0[s]);
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      if (ok && item.ntile[s] > 0) {
+        ok = __all_sync(FULL, wait_bar(sm.q_empty(s), (q_uses[s] & 1) ^ 1, ctl));
+        ++q_uses[s];
+        if (ok && ptx::elect_one()) {
+          ptx::mbar_arrive_expect_tx(sm.q_full(s), C::kQTile);
+          for (int c = 0; c < C::kChunks; ++c)
+            ptx::tma_load_3d(sm.q(s) + c * C::kQChunk, tm_q, sm.q_full(s), c * 64, item.head[s],
+                             item.q_row0[s]);
+        }
+        __syncwarp();
       }
-      __syncwarp();
     }
     const int n = max(item.ntile[0], item.ntile[1]);
     for (int j = 0; j < n && ok; ++j) {
@@ -257,51 +259,69 @@ __device__ void load_role(const Smem<D>& sm, const CUtensorMap* tm_q, const CUte
       drain_bar(sm.kv_full(st), (uses - 1) & 1);
     }
   }
+#pragma unroll
   for (int s = 0; s < 2; ++s)
     if (q_uses[s] > 0) drain_bar(sm.q_full(s), (q_uses[s] - 1) & 1);
 }
 
 // ------------------------------------------------------------------ MMA issue
+// The MMA warp issues 32 tensor-core instructions per pair of slot tiles, so
+// their operands are prepared once: a descriptor's start-address field holds
+// the shared-memory byte address / 16 (14 bits, and every address of the CTA
+// is below 2^18), so a descriptor of base + off is the base's descriptor +
+// off / 16. The loops below add compile-time offsets only.
+struct MmaDescs {
+  uint64_t q[2];   // Q of slot s, chunk 0, K-major
+  uint64_t k0;     // K ring stage 0, chunk 0, K-major
+  uint64_t v0;     // V ring stage 0, MN-major
+};
+
+template <int D>
+__device__ __forceinline__ uint64_t stage_desc(uint64_t d0, int st) {
+  return d0 + (uint64_t)(st * (KCfg<D>::kKVTile >> 4));
+}
+
 // S_s = Q_s K^T: M = 128, N = 128 keys, K = D in steps of 16.
 template <int D>
-__device__ __forceinline__ void issue_s(const Smem<D>& sm, uint32_t tmem, int s, int kst) {
+__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t qd, uint64_t kd) {
   using C = KCfg<D>;
+  static_assert(C::kQChunk == C::kKVChunk, "Q and K chunks share the offsets");
   constexpr uint32_t idesc = idesc_bf16(BN, false);
-  const uint32_t qa = ptx::smem_u32(sm.q(s));
-  const uint32_t ka = ptx::smem_u32(sm.kv(kst));
 #pragma unroll
   for (int k16 = 0; k16 < D / 16; ++k16) {
-    const uint32_t in = (k16 & 3) * 32;
-    ptx::mma_ss(tmem + s_col(s), desc_kmajor_sw128(qa + (k16 >> 2) * C::kQChunk + in),
-                desc_kmajor_sw128(ka + (k16 >> 2) * C::kKVChunk + in), idesc, k16 > 0);
+    const uint64_t off = (uint64_t)((((k16 >> 2) * C::kQChunk) + (k16 & 3) * 32) >> 4);
+    ptx::mma_ss(d_tmem, qd + off, kd + off, idesc, k16 > 0 ? 1u : 0u);
   }
 }
 
 // O_s += P_s[keys 64h .. 64h+63] V[same keys]: M = 128, N = D, K = 64 in
 // steps of 16; P from tensor memory (2 keys per 32-bit column).
 template <int D>
-__device__ __forceinline__ void issue_pv_half(const Smem<D>& sm, uint32_t tmem, int s, int h,
-                                              int vst, bool acc) {
-  using C = KCfg<D>;
+__device__ __forceinline__ void issue_pv_half(uint32_t o_tmem, uint32_t p_tmem, uint64_t vd, int h,
+                                              bool acc) {
   constexpr uint32_t idesc = idesc_bf16(D, true);
-  const uint32_t va = ptx::smem_u32(sm.kv(vst));
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int k16 = 4 * h + k;
-    ptx::mma_ts(tmem + o_col<D>(s), tmem + s_col(s) + k16 * 8,
-                desc_mnmajor_sw128(va + k16 * 16 * 128, C::kKVChunk), idesc,
+    ptx::mma_ts(o_tmem, p_tmem + k16 * 8, vd + (uint64_t)((k16 * 16 * 128) >> 4), idesc,
                 (acc || k16 > 0) ? 1u : 0u);
   }
 }
 
 // Runs on all 32 lanes of the MMA warp (uniform control flow); one elected
-// lane issues the tensor-core instructions and their commits.
+// lane issues the tensor-core instructions and their commits. The slot loops
+// are unrolled so that every per-slot counter stays in a register.
 template <int D>
 __device__ void mma_role(const Smem<D>& sm, uint32_t tmem, const Ctl& ctl) {
   using C = KCfg<D>;
   const unsigned FULL = 0xffffffffu;
   uint32_t kv_t = 0, q_uses[2] = {0, 0}, o_uses[2] = {0, 0};
   uint32_t tc[2] = {0, 0};  // tiles issued per slot (phase of the P barriers)
+  MmaDescs dsc;
+  dsc.q[0] = desc_kmajor_sw128(ptx::smem_u32(sm.q(0)));
+  dsc.q[1] = desc_kmajor_sw128(ptx::smem_u32(sm.q(1)));
+  dsc.k0 = desc_kmajor_sw128(ptx::smem_u32(sm.kv(0)));
+  dsc.v0 = desc_mnmajor_sw128(ptx::smem_u32(sm.kv(0)), C::kKVChunk);
   auto wait = [&](uint64_t* bar, uint32_t parity) {
     return __all_sync(FULL, wait_bar(bar, parity, ctl));
   };
@@ -315,18 +335,21 @@ __device__ void mma_role(const Smem<D>& sm, uint32_t tmem, const Ctl& ctl) {
   for (int it = 0; ok; ++it) {
     const int k = it & 1;
     if (!wait(sm.item_full(k), (it >> 1) & 1)) break;
-    const Item item = sm.items()[k];
+    const Item& itm = sm.items()[k];
+    const int valid = itm.valid;
+    const int nt[2] = {itm.ntile[0], itm.ntile[1]};
     __syncwarp();
     if (ptx::elect_one()) ptx::mbar_arrive(sm.item_empty(k));
-    if (!item.valid) break;
-    const int nt[2] = {item.ntile[0], item.ntile[1]};
+    if (!valid) break;
     const int n = max(nt[0], nt[1]);
     if (n == 0) continue;
-    for (int s = 0; s < 2 && ok; ++s)
-      if (nt[s] > 0) {
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      if (ok && nt[s] > 0) {
         ok = wait(sm.q_full(s), q_uses[s] & 1);
         ++q_uses[s];
       }
+    }
     if (!ok) break;
     // K0 and the first scores
     {
@@ -334,11 +357,14 @@ __device__ void mma_role(const Smem<D>& sm, uint32_t tmem, const Ctl& ctl) {
       if (!next_kv(kst)) break;
       ptx::tc_fence_after();
       if (ptx::elect_one()) {
+        const uint64_t kd = stage_desc<D>(dsc.k0, kst);
+#pragma unroll
         for (int s = 0; s < 2; ++s) {
-          if (nt[s] <= 0) continue;
-          issue_s<D>(sm, tmem, s, kst);
-          ptx::tc_commit(sm.s_full(s));
-          if (nt[s] == 1) ptx::tc_commit(sm.q_empty(s));
+          if (nt[s] > 0) {
+            issue_s<D>(tmem + s_col(s), dsc.q[s], kd);
+            ptx::tc_commit(sm.s_full(s));
+            if (nt[s] == 1) ptx::tc_commit(sm.q_empty(s));
+          }
         }
         ptx::tc_commit(sm.kv_empty(kst));
       }
@@ -347,36 +373,42 @@ __device__ void mma_role(const Smem<D>& sm, uint32_t tmem, const Ctl& ctl) {
     for (int j = 0; j < n && ok; ++j) {
       int vst;
       if (!next_kv(vst)) { ok = false; break; }
+      const uint64_t vd = stage_desc<D>(dsc.v0, vst);
       int kst = -1;
+#pragma unroll
       for (int s = 0; s < 2; ++s) {
-        if (j < nt[s]) {
+        if (ok && j < nt[s]) {
           const uint32_t ph = (tc[s] + j) & 1;
           if (j == 0) {
-            if (!wait(sm.o_empty(s), (o_uses[s] & 1) ^ 1)) { ok = false; break; }
+            ok = wait(sm.o_empty(s), (o_uses[s] & 1) ^ 1);
             ++o_uses[s];
           }
+#pragma unroll
           for (int h = 0; h < 2; ++h) {
-            if (!wait(sm.p_full(s, h), ph)) { ok = false; break; }
+            if (ok) ok = wait(sm.p_full(s, h), ph);
+            if (ok) {
+              ptx::tc_fence_after();
+              if (ptx::elect_one()) {
+                issue_pv_half<D>(tmem + o_col<D>(s), tmem + s_col(s), vd, h, j > 0);
+                if (h == 1 && j == nt[s] - 1) ptx::tc_commit(sm.o_full(s));
+              }
+              __syncwarp();
+            }
+          }
+        }
+        if (ok && j + 1 < nt[s]) {
+          if (kst < 0) {
+            ok = next_kv(kst);
             ptx::tc_fence_after();
+          }
+          if (ok) {
             if (ptx::elect_one()) {
-              issue_pv_half<D>(sm, tmem, s, h, vst, j > 0);
-              if (h == 1 && j == nt[s] - 1) ptx::tc_commit(sm.o_full(s));
+              issue_s<D>(tmem + s_col(s), dsc.q[s], stage_desc<D>(dsc.k0, kst));
+              ptx::tc_commit(sm.s_full(s));
+              if (j + 2 == nt[s]) ptx::tc_commit(sm.q_empty(s));
             }
             __syncwarp();
           }
-          if (!ok) break;
-        }
-        if (j + 1 < nt[s]) {
-          if (kst < 0) {
-            if (!next_kv(kst)) { ok = false; break; }
-            ptx::tc_fence_after();
-          }
-          if (ptx::elect_one()) {
-            issue_s<D>(sm, tmem, s, kst);
-            ptx::tc_commit(sm.s_full(s));
-            if (j + 2 == nt[s]) ptx::tc_commit(sm.q_empty(s));
-          }
-          __syncwarp();
         }
       }
       if (!ok) break;
@@ -428,21 +460,29 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
     const int k = it & 1;
     ok = __all_sync(FULL, wait_bar(sm.item_full(k), (it >> 1) & 1, ctl));
     if (!ok) break;
-    const Item item = sm.items()[k];
+    // This slot's fields, read from shared memory (a local copy of the item
+    // indexed by the warp-dependent slot would live in local memory).
+    const Item& itm = sm.items()[k];
+    const int valid = itm.valid;
+    const int rows = itm.rows[wg];
+    const int n = itm.ntile[wg];
+    const int head = itm.head[wg];
+    const int q_loc0 = itm.q_loc0[wg];
+    const int q_row0 = itm.q_row0[wg];
+    const int seq = itm.seq;
+    const int Lq = itm.Lq;
+    const int Lk = itm.Lk;
+    const int kv_row0 = itm.kv_row0;
     __syncwarp();
     if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(sm.item_empty(k));
-    if (!item.valid) break;
-    const int rows = item.rows[wg];
+    if (!valid) break;
     if (rows == 0) continue;
-    const int n = item.ntile[wg];
-    const int head = item.head[wg];
-    const int q_loc = item.q_loc0[wg] + r;
+    const int q_loc = q_loc0 + r;
     const bool row_ok = r < rows;
-    const int Lk = item.Lk;
-    const int limit = p.causal ? min(Lk, q_loc + (Lk - item.Lq) + 1) : Lk;
+    const int limit = p.causal ? min(Lk, q_loc + (Lk - Lq) + 1) : Lk;
     const float* brow = nullptr;
     if (kBiasPair && row_ok)
-      brow = p.bias_pair + (long long)item.seq * p.sb + (long long)head * p.sh +
+      brow = p.bias_pair + (long long)seq * p.sb + (long long)head * p.sh +
              (long long)q_loc * p.sr;
     float m_used = -INFINITY, l = 0.f;
 
@@ -455,7 +495,7 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
       if constexpr (kBiasKey) {
         bk = sm.bias(wg, b);
         const int key = kb + r;
-        bk[r] = key < Lk ? p.bias_key[(long long)(item.kv_row0 + key) * p.n_heads + head] * kLog2e
+        bk[r] = key < Lk ? p.bias_key[(long long)(kv_row0 + key) * p.n_heads + head] * kLog2e
                          : 0.f;
         ptx::mbar_arrive(sm.bias_full(wg, b));
       }
@@ -587,7 +627,7 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
     }
     const float inv = l > 0.f ? 1.f / l : 0.f;
     __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) +
-                          ((long long)(item.q_row0[wg] + r) * p.n_heads + head) * D;
+                          ((long long)(q_row0 + r) * p.n_heads + head) * D;
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
       uint32_t o[32];
@@ -615,7 +655,7 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
     }
     if (row_ok && p.lse != nullptr) {
       const float lse = l > 0.f ? (m_used + __log2f(l)) * kLn2 : -INFINITY;
-      p.lse[(long long)head * p.total_q + item.q_row0[wg] + r] = lse;
+      p.lse[(long long)head * p.total_q + q_row0 + r] = lse;
     }
   }
 }
@@ -644,7 +684,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ptx::mbar_init(sm.o_full(s), 1);
       ptx::mbar_init(sm.o_empty(s), 128);
       ptx::mbar_init(sm.item_full(s), 1);
-      ptx::mbar_init(sm.item_empty(s), 1 + 8);
+      ptx::mbar_init(sm.item_empty(s), 1 + 8);  // MMA warp, eight softmax warps
     }
     ptx::mbar_init(sm.drain(), 1);
     for (int st = 0; st < KCfg<D>::kStages; ++st) {

@@ -96,6 +96,7 @@ __host__ __device__ __forceinline__ int seq_groups(int Lq, int pairing) {
 
 __device__ __forceinline__ void fill_slots(Item& it, int g, int hg, int pairing, int group,
                                            int n_hp, int causal) {
+#pragma unroll
   for (int s = 0; s < 2; ++s) {
     int active, head, q_loc0;
     if (pairing == kPairHeads) {

@@ -7,11 +7,16 @@
 //      error word gets kErrBadSeqlens and the work count is 0, so the
 //      attention kernel does nothing and reads nothing out of range;
 //   2. enumerate the (sequence, group) pairs with a block-wide prefix sum;
-//   3. sort them by K/V tiles to visit, descending (ties by position in the
-//      stream), with an in-shared-memory bitonic sort of 64-bit keys;
+//   3. order them with an in-shared-memory bitonic sort of 64-bit keys:
+//      sequences by size, largest first, and within a sequence the pairs by
+//      K/V tiles to visit, descending (ties by position in the stream);
 //   4. publish the list, the item count and a zeroed fetch counter.
 // Each pair expands to n_hg consecutive work items (head groups), so the
 // heads of one q-block run side by side and share K/V and bias tiles in L2.
+// Grouping by sequence keeps the CTAs that run at the same time on the K/V
+// of one sequence (a few tens of MB at most), which then stays in L2
+// instead of being fetched from HBM again for every q-block; largest first
+// within and across sequences keeps the longest items away from the end.
 #pragma once
 #include "common.cuh"
 
@@ -19,6 +24,7 @@ namespace va {
 
 constexpr int kSchedThreads = 1024;
 constexpr int kSortCap = 8192;  // pairs sorted in shared memory; beyond: stream order
+static_assert(kSortCap <= (1 << 20), "stream position must fit the low 20 bits of a sort key");
 
 __device__ __forceinline__ int block_exclusive_scan(int x, int* warp_sums, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -129,7 +135,13 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedParams 
           rows = rows < 0 ? 0 : (rows > BM ? BM : rows);
           work += slot_tiles(q_loc0, rows, it.Lq, it.Lk, p.causal);
         }
-        key = ((unsigned long long)(0x7fffffff - work) << 32) | (unsigned)k;
+        // key: [63:40] sequence size (descending), [39:20] item work
+        // (descending), [19:0] stream position (k < kSortCap <= 2^20).
+        long long sk = (long long)ceil_div(it.Lq, BM) * ceil_div(it.Lk, BN);
+        sk = sk > 0xFFFFFF ? 0xFFFFFF : sk;
+        const int wk = work > 0xFFFFF ? 0xFFFFF : work;
+        key = ((unsigned long long)(0xFFFFFF - sk) << 40) |
+              ((unsigned long long)(0xFFFFF - wk) << 20) | (unsigned)k;
       }
       sort_keys[k] = key;
     }
@@ -151,7 +163,7 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedParams 
       }
     }
     for (int k = tid; k < P; k += kSchedThreads)
-      p.ws.list[k] = p.ws.tmp[(int)(sort_keys[k] & 0xffffffffu)];
+      p.ws.list[k] = p.ws.tmp[(int)(sort_keys[k] & 0xFFFFFu)];
   } else {
     for (int k = tid; k < P; k += kSchedThreads) p.ws.list[k] = p.ws.tmp[k];
   }
