@@ -123,11 +123,13 @@ class ClockSampler:
                 return None
         sm = [num(r[1]) for r in self.rows if num(r[1]) is not None]
         mx = [num(r[2]) for r in self.rows if num(r[2]) is not None]
+        pw = [num(r[3]) for r in self.rows if num(r[3]) is not None]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in self.rows for i in range(4)
                           if r[5 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "power_w": statistics.median(pw) if pw else None,
                 "samples": len(self.rows)}
 
 
@@ -346,7 +348,7 @@ def run_gpu(args, world, rank, local):
         value = all_flops / (ms_per_step * 1e-3) / 1e12
         achieved = flops / (kern_ms * 1e-3) / 1e12  # this rank's kernel, per launch
         peak = float(peaks["bf16_tflops"])
-        traffic = _profiled_traffic()
+        traffic = _profiled_traffic() if not args.sequences else None  # profiled on the full workload
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,

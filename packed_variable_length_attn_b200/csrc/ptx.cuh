@@ -201,41 +201,10 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
-__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
-}
-
-// 2^x for a pair of fp32 values on the FMA pipe instead of the XU pipe.
-// x is clamped to >= -127 and split as x = n + f with n = round(x) (the
-// 1.5 * 2^23 rounding trick) and f in [-1/2, 1/2]; 2^f comes from a degree-3
-// polynomial fitted by relative-error minimax (Remez exchange; the fit and
-// its error, 7.5e-5 relative, are reproduced by csrc/exp2_poly_fit.py) and
-// 2^n is built from its exponent bits. n = -127 gives 2^n = +0, so masked
-// (-inf) scores give exactly 0. Requires x <= 127.
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  float x0, x1;
-  f2_split(x, x0, x1);
-  x = f2(fmaxf(x0, -127.0f), fmaxf(x1, -127.0f));
-  const uint64_t y = fadd2(x, f2(kRound, kRound));
-  const uint64_t nf = fadd2(y, f2(-kRound, -kRound));
-  const uint64_t f = ffma2(nf, f2(-1.0f, -1.0f), x);
-  uint64_t q = ffma2(f, f2(5.517166853e-02f, 5.517166853e-02f), f2(2.426111251e-01f, 2.426111251e-01f));
-  q = ffma2(q, f, f2(6.932609677e-01f, 6.932609677e-01f));
-  q = ffma2(q, f, f2(9.999280572e-01f, 9.999280572e-01f));
-  float y0, y1;
-  f2_split(y, y0, y1);
-  // bits(y) = bits(1.5 * 2^23) + n, and bits(1.5 * 2^23) << 23 wraps to 0.
-  const float s0 = __uint_as_float((__float_as_uint(y0) << 23) + 0x3F800000u);
-  const float s1 = __uint_as_float((__float_as_uint(y1) << 23) + 0x3F800000u);
-  return fmul2(q, f2(s0, s1));
 }
 
 // Register reallocation between warpgroups (all 128 threads execute it).
