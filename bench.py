@@ -238,6 +238,31 @@ def _config(w):
             "l2": f"inputs larger than L2 (Q+K+V {qkv_bytes / 1e9:.2f} GB > 126 MB); no flush"}
 
 
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own batch of the workload (weak scaling)."""
+    from packed_variable_length_attn_b200 import workloads
+    return workloads.SEED_BASE + WORKLOAD + 1000 * rank
+
+
+def reduce_over_ranks(stats, totals, world, device=None):
+    """MAX over ranks of the times [timed ms, end-to-end ms, kernel ms] (the
+    job is as slow as its slowest rank) and SUM of the work [FLOPs, tokens].
+    The only collectives of the benchmark; every rank calls this once."""
+    import torch
+    import torch.distributed as dist
+    s = torch.tensor(list(stats), dtype=torch.float64, device=device)
+    t = torch.tensor(list(totals), dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(s, op=dist.ReduceOp.MAX)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return s.tolist(), t.tolist()
+
+
+def throughput_tflops(all_flops: float, ms_per_step: float) -> float:
+    """Whole-job useful TFLOP/s: the FLOPs of all ranks over the slowest rank's time."""
+    return all_flops / (ms_per_step * 1e-3) / 1e12
+
+
 def run_gpu(args, world, rank, local):
     import torch
     import torch.distributed as dist
@@ -248,8 +273,7 @@ def run_gpu(args, world, rank, local):
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
-    seed = workloads.SEED_BASE + WORKLOAD + 1000 * rank
-    w = _workload(args, seed=seed)
+    w = _workload(args, seed=rank_seed(rank))
     flops = metrics.useful_flops(w.lengths_q, w.lengths_k, w.causal, w.n_heads, w.head_dim)
     dev = torch.device("cuda", local)
     q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
@@ -333,19 +357,14 @@ def run_gpu(args, world, rank, local):
     d2h = hout.numel() * hout.element_size() + hlse.numel() * hlse.element_size()
 
     # ---- reduce over ranks
-    stats = torch.tensor([elapsed_ms, e2e_ms, sum(kernel_ms) / len(kernel_ms)],
-                         dtype=torch.float64, device=dev)
-    tot = torch.tensor([float(flops), float(w.total_q)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
-        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
-    elapsed_ms, e2e_ms, kern_ms = stats.tolist()
-    all_flops, all_tokens = tot.tolist()
+    (elapsed_ms, e2e_ms, kern_ms), (all_flops, all_tokens) = reduce_over_ranks(
+        [elapsed_ms, e2e_ms, sum(kernel_ms) / len(kernel_ms)], [float(flops), float(w.total_q)],
+        world, device=dev)
 
     if rank == 0:
         peaks, peak_src = _peaks()
         ms_per_step = elapsed_ms / args.steps
-        value = all_flops / (ms_per_step * 1e-3) / 1e12
+        value = throughput_tflops(all_flops, ms_per_step)
         achieved = flops / (kern_ms * 1e-3) / 1e12  # this rank's kernel, per launch
         peak = float(peaks["bf16_tflops"])
         traffic = _profiled_traffic() if not args.sequences else None  # profiled on the full workload
@@ -363,7 +382,7 @@ def run_gpu(args, world, rank, local):
                          "frac_of_sustained": achieved / float(peaks["bf16_tflops_sustained"]),
                          "kernel": "attn_fwd_sm100<128,false,false>",
                          "kernel_ms_per_launch": kern_ms},
-            "e2e": {"value": all_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": throughput_tflops(all_flops, e2e_ms), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms, "steps": e_steps},
             "gpu_launches": va.launches_per_call() * args.steps,
