@@ -579,8 +579,8 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
       const float mb = m_used == -INFINITY ? 0.f : m_used;
       // P = 2^(s * sfac - mb): one packed FMA per pair, one XU ex2 per score.
       // (Moving part of the exponentials to an FMA-pipe polynomial balanced
-      // the pipes but added about ten instructions per pair; the kernel runs
-      // at the power cap, where fewer instructions per score win: all-ex2
+      // the pipes but added about ten instructions per pair; under load the
+      // clock is held well below its maximum (sw_power_cap), and all-ex2
       // measured 12-14% faster.) Each half of the keys is stored and
       // published as soon as it is ready.
       const uint64_t sf2 = ptx::f2(sfac, sfac), nm2 = ptx::f2(-mb, -mb);
