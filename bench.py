@@ -6,6 +6,12 @@ lengths U[2048, 8192], 32 query / 8 K/V heads, head_dim 128, causal), inputs
 already resident in HBM. The batch is seeded and synthetic.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--config 1..5] [--flush-l2]
+
+``--config`` times one of the other named workloads instead (the parity-test
+configurations: tiny packed causal, GenRec prompts, graph batch with pair and
+per-key biases, short-query GQA); ``--flush-l2`` writes a 256 MB scrub buffer
+between timed steps and times each call with its own events.
 
 Prints one JSON line (rank 0). Under torchrun every rank runs its own batch
 (weak scaling: per-GPU work fixed, no data-path collective); the time is the
@@ -29,7 +35,14 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "varlen attn fwd useful TFLOP/s & tokens/s on 1 B200; % of bf16 tensor peak"
-WORKLOAD = 5
+WORKLOAD = 5            # the long causal GQA workload; --config picks another
+# Per workload: what bounds the kernel, and how its inputs were drawn.
+BOUND = {1: "tensor", 2: "tensor", 3: "hbm", 4: "hbm", 5: "tensor"}
+LENGTHS = {1: "fixed {5, 17, 32, 64}", 2: "uniform [128, 2048]", 3: "uniform [1, 256]",
+           4: "fixed Lq 112, Lk 262", 5: "uniform [2048, 8192]"}
+BIAS = {3: "pair grid fp32 [512,1,256,256] N(0,1), strides (65536,0,256,1); "
+           "per-key fp32 [Tk,8] N(0,0.5)"}
+L2_SCRUB_BYTES = 256 << 20
 KERNEL_SOURCES = ["attn_sm100.cuh", "ptx.cuh", "common.cuh"]
 PROFILE_FILE = os.path.join(ROOT, "profiles", "attn_fwd_sm100_long_causal_gqa.md")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -142,14 +155,16 @@ def _dist():
 
 def _workload(args, seed=None):
     from packed_variable_length_attn_b200 import workloads
-    w = workloads.make(WORKLOAD, seed=seed)
+    w = workloads.make(getattr(args, "config", WORKLOAD), seed=seed)
     if args.sequences and args.sequences < w.batch:
         n = args.sequences
         tq, tk = int(w.cu_q[n]), int(w.cu_k[n])
         w = workloads.Workload(f"{w.name}_first{n}", w.lengths_q[:n], w.lengths_k[:n],
                                w.cu_q[:n + 1].clone(), w.cu_k[:n + 1].clone(), w.q[:tq].clone(),
                                w.k[:tk].clone(), w.v[:tk].clone(), w.n_heads, w.n_kv_heads,
-                               w.head_dim, w.causal, w.softmax_scale, meta=dict(w.meta))
+                               w.head_dim, w.causal, w.softmax_scale,
+                               None if w.bias_key is None else w.bias_key[:tk].clone(),
+                               w.bias_pair, w.bias_strides, meta=dict(w.meta))
     return w
 
 
@@ -176,7 +191,7 @@ def run_reference(args, world, rank):
         "n_gpus": world, "steps": steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * secs / steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-        "config": _config(w),
+        "config": _config(w, args),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res["cores"],
                          "kind": "oracle",
                          "sample": f"{res['n_rows']} random (sequence, head, query row) outputs "
@@ -212,7 +227,9 @@ def oracle_sample_rate(w, budget_s=None, n_rows=None, seed=0):
         seq, head, row = pick(n)
         t0 = time.perf_counter()
         oracle.rows(w.q, w.k, w.v, w.cu_q, w.cu_k, w.n_heads, w.n_kv_heads, w.softmax_scale,
-                    w.causal, seq, head, row, threads=cores)
+                    w.causal, seq, head, row, bias_key=w.bias_key, bias_pair=w.bias_pair,
+                    bias_strides=w.bias_strides if w.bias_pair is not None else None,
+                    threads=cores)
         return flops_of(seq, row), time.perf_counter() - t0
 
     if n_rows is None:
@@ -226,22 +243,30 @@ def oracle_sample_rate(w, budget_s=None, n_rows=None, seed=0):
     return {"flops": f, "seconds": s, "n_rows": n_rows, "cores": cores}
 
 
-def _config(w):
+def _config(w, args=None):
     from packed_variable_length_attn_b200 import metrics
+    cfg = getattr(args, "config", WORKLOAD)
     pairs = metrics.useful_pairs(w.lengths_q, w.lengths_k, w.causal)
     qkv_bytes = (w.q.numel() + w.k.numel() + w.v.numel()) * 2
-    return {"workload": w.name, "sequences": w.batch, "lengths": "uniform [2048, 8192]",
-            "lengths_drawn": list(w.lengths_q),
-            "total_tokens": w.total_q, "n_heads": w.n_heads, "n_kv_heads": w.n_kv_heads,
-            "head_dim": w.head_dim, "causal": w.causal, "bias": None,
-            "useful_pairs_per_head": pairs, "seed": w.meta.get("seed"),
-            "l2": f"inputs larger than L2 (Q+K+V {qkv_bytes / 1e9:.2f} GB > 126 MB); no flush"}
+    if getattr(args, "flush_l2", False):
+        l2 = f"L2 flushed: {L2_SCRUB_BYTES >> 20} MB scrub write between timed steps"
+    elif qkv_bytes > 126e6:
+        l2 = f"inputs larger than L2 (Q+K+V {qkv_bytes / 1e9:.2f} GB > 126 MB); no flush"
+    else:
+        l2 = f"hot L2 (Q+K+V {qkv_bytes / 1e6:.1f} MB; no flush)"
+    d = {"workload": w.name, "sequences": w.batch, "lengths": LENGTHS[cfg],
+         "total_tokens": w.total_q, "n_heads": w.n_heads, "n_kv_heads": w.n_kv_heads,
+         "head_dim": w.head_dim, "causal": w.causal, "bias": BIAS.get(cfg),
+         "useful_pairs_per_head": pairs, "seed": w.meta.get("seed"), "l2": l2}
+    if w.batch <= 64:
+        d["lengths_drawn"] = list(w.lengths_q)
+    return d
 
 
-def rank_seed(rank: int) -> int:
+def rank_seed(rank: int, config: int = WORKLOAD) -> int:
     """Each rank draws its own batch of the workload (weak scaling)."""
     from packed_variable_length_attn_b200 import workloads
-    return workloads.SEED_BASE + WORKLOAD + 1000 * rank
+    return workloads.SEED_BASE + config + 1000 * rank
 
 
 def reduce_over_ranks(stats, totals, world, device=None):
@@ -273,18 +298,23 @@ def run_gpu(args, world, rank, local):
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
-    w = _workload(args, seed=rank_seed(rank))
+    w = _workload(args, seed=rank_seed(rank, args.config))
     flops = metrics.useful_flops(w.lengths_q, w.lengths_k, w.causal, w.n_heads, w.head_dim)
     dev = torch.device("cuda", local)
     q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
     cu_q, cu_k = w.cu_q.to(dev), w.cu_k.to(dev)
     out = torch.empty_like(q)
     lse = torch.empty((w.n_heads, w.total_q), dtype=torch.float32, device=dev)
+    bias_kw = dict(
+        bias_per_key=None if w.bias_key is None else w.bias_key.to(dev),
+        bias_pair=None if w.bias_pair is None else w.bias_pair.to(dev),
+        bias_pair_strides=w.bias_strides if w.bias_pair is not None else None)
     stream = torch.cuda.current_stream()
 
     def step():
         va.varlen_attn_fwd(q, k, v, cu_q, cu_k, w.max_seqlen_q, w.max_seqlen_k,
-                           softmax_scale=w.softmax_scale, causal=True, out=out, lse=lse)
+                           softmax_scale=w.softmax_scale, causal=w.causal, out=out, lse=lse,
+                           **bias_kw)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -306,17 +336,33 @@ def run_gpu(args, world, rank, local):
     time.sleep(0.3)  # let the sampler start before the timed region
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for i in range(args.steps):
-        va.set_profile_events(*kev[i])
-        step()
-    va.set_profile_events()
-    t1.record(stream)
+    if args.flush_l2:
+        # each call timed on its own, a scrub write larger than L2 between calls
+        scrub = torch.empty(L2_SCRUB_BYTES // 4, dtype=torch.float32, device=dev)
+        cev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for i in range(args.steps):
+            scrub.fill_(float(i))
+            cev[i][0].record(stream)
+            va.set_profile_events(*kev[i])
+            step()
+            va.set_profile_events()
+            cev[i][1].record(stream)
+    else:
+        t0.record(stream)
+        for i in range(args.steps):
+            va.set_profile_events(*kev[i])
+            step()
+        va.set_profile_events()
+        t1.record(stream)
     torch.cuda.synchronize()
     sampler.stop()
     if world > 1:
         dist.barrier()
-    elapsed_ms = t0.elapsed_time(t1)
+    if args.flush_l2:
+        elapsed_ms = sum(a.elapsed_time(b) for a, b in cev)
+    else:
+        elapsed_ms = t0.elapsed_time(t1)
     kernel_ms = [a.elapsed_time(b) for a, b in kev]
     if va.get_device_error() != 0:
         raise RuntimeError("device error during the timed region")
@@ -336,7 +382,8 @@ def run_gpu(args, world, rank, local):
         dcq.copy_(hcq, non_blocking=True)
         dck.copy_(hck, non_blocking=True)
         va.varlen_attn_fwd(dq, dk_, dv, dcq, dck, w.max_seqlen_q, w.max_seqlen_k,
-                           softmax_scale=w.softmax_scale, causal=True, out=out, lse=lse)
+                           softmax_scale=w.softmax_scale, causal=w.causal, out=out, lse=lse,
+                           **bias_kw)
         hout.copy_(out, non_blocking=True)
         hlse.copy_(lse, non_blocking=True)
 
@@ -367,21 +414,36 @@ def run_gpu(args, world, rank, local):
         value = throughput_tflops(all_flops, ms_per_step)
         achieved = flops / (kern_ms * 1e-3) / 1e12  # this rank's kernel, per launch
         peak = float(peaks["bf16_tflops"])
-        traffic = _profiled_traffic() if not args.sequences else None  # profiled on the full workload
+        # profiled on the full long workload only
+        traffic = (_profiled_traffic()
+                   if not args.sequences and args.config == WORKLOAD and not args.flush_l2
+                   else None)
+        bound = BOUND[args.config]
+        if bound == "hbm":
+            abytes = metrics.algorithmic_bytes(w)
+            rl = {"bound": "hbm", "achieved": abytes / (kern_ms * 1e-3) / 1e9,
+                  "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                  "algorithmic_bytes_per_launch": abytes,
+                  "peak_source": f"{peak_src} hbm_gbs",
+                  "tflops_per_launch": flops / (kern_ms * 1e-3) / 1e12}
+        else:
+            rl = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                  "peak_source": f"{peak_src} bf16_tflops (burst)",
+                  "frac_of_sustained": achieved / float(peaks["bf16_tflops_sustained"])}
+        rl["frac"] = rl["achieved"] / rl["peak"]
+        rl["traffic"] = traffic
+        rl["kernel"] = (f"attn_fwd_sm100<{w.head_dim},{str(w.bias_key is not None).lower()},"
+                        f"{str(w.bias_pair is not None).lower()}>")
+        rl["kernel_ms_per_launch"] = kern_ms
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded N(0,1) bf16 Q/K/V; lengths uniform [2048, 8192])",
-            "config": _config(w),
+            "data": f"synthetic (seeded N(0,1) bf16 Q/K/V; lengths {LENGTHS[args.config]})",
+            "config": _config(w, args),
             "tokens_per_s": all_tokens / (ms_per_step * 1e-3),
             "pct_of_bf16_peak": 100.0 * value / (peak * world),
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": f"{peak_src} bf16_tflops (burst)",
-                         "frac_of_sustained": achieved / float(peaks["bf16_tflops_sustained"]),
-                         "kernel": "attn_fwd_sm100<128,false,false>",
-                         "kernel_ms_per_launch": kern_ms},
+            "roofline": rl,
             "e2e": {"value": throughput_tflops(all_flops, e2e_ms), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms, "steps": e_steps},
@@ -413,6 +475,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-total-s", type=float, default=150.0,
                     help="--impl reference: seconds of oracle work over all steps")
+    ap.add_argument("--config", type=int, default=WORKLOAD, choices=[1, 2, 3, 4, 5],
+                    help="named workload (default: the long causal GQA workload)")
+    ap.add_argument("--flush-l2", action="store_true",
+                    help="256 MB scrub write between timed steps; each call timed alone")
     ap.add_argument("--sequences", type=int, default=0,
                     help="use only the first N sequences (small case for profiling)")
     args = ap.parse_args()

@@ -43,3 +43,22 @@ def useful_pairs(lengths_q: Sequence[int], lengths_k: Sequence[int], causal: boo
 
 def useful_flops(lengths_q, lengths_k, causal, n_heads, head_dim) -> int:
     return 4 * int(head_dim) * int(n_heads) * useful_pairs(lengths_q, lengths_k, causal)
+
+
+def algorithmic_bytes(w) -> int:
+    """Bytes one forward must move at least: Q, K, V read once (bf16), O
+    written once (bf16), LSE written (fp32 [Hq, Tq]), the per-key bias read
+    once (fp32 [Tk, Hq]) and, of the per-pair grid, only the in-sequence
+    entries (Lq_i x Lk_i per sequence, per head unless the grid broadcasts
+    heads), read once."""
+    e = 2  # bf16
+    tq, tk = w.total_q, w.total_k
+    b = tq * w.n_heads * w.head_dim * e * 2             # Q read, O written
+    b += 2 * tk * w.n_kv_heads * w.head_dim * e         # K, V
+    b += tq * w.n_heads * 4                              # LSE
+    if w.bias_key is not None:
+        b += tk * w.n_heads * 4
+    if w.bias_pair is not None:
+        heads = 1 if w.bias_strides[1] == 0 else w.n_heads
+        b += 4 * heads * sum(int(lq) * int(lk) for lq, lk in zip(w.lengths_q, w.lengths_k))
+    return b

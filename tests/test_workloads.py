@@ -40,3 +40,16 @@ def test_determinism():
     b = workloads.make(2)
     assert a.lengths_q == b.lengths_q
     assert torch.equal(a.q.view(torch.int16), b.q.view(torch.int16))
+
+
+def test_algorithmic_bytes_closed_forms():
+    """Bytes one forward must move, checked against closed forms."""
+    from packed_variable_length_attn_b200 import metrics, workloads
+    w4 = workloads.make(4)  # 64 rows of 112 queries, 262 keys, 32/8 heads, D 128
+    want = 64 * 112 * 32 * 128 * 2 * 2 + 2 * 64 * 262 * 8 * 128 * 2 + 64 * 112 * 32 * 4
+    assert metrics.algorithmic_bytes(w4) == want
+    w3 = workloads.make(3)  # one-head pair grid (heads broadcast) + per-key bias
+    base = (w3.total_q * 8 * 64 * 2 * 2 + 2 * w3.total_k * 8 * 64 * 2 + w3.total_q * 8 * 4
+            + w3.total_k * 8 * 4)
+    grid = 4 * sum(L * L for L in w3.lengths_q)
+    assert metrics.algorithmic_bytes(w3) == base + grid
