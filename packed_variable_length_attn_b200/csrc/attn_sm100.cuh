@@ -29,7 +29,8 @@
 //
 // Shared memory: Q0, Q1 (128 rows x D bf16, 64-column 128-byte-swizzled
 // chunks as TMA writes them), the K/V ring (128-row tiles, same layout),
-// per-key bias staging, the work-item ring, mbarriers.
+// per-key bias staging, O staging for coalesced output stores, the
+// work-item ring, mbarriers.
 //
 // Every mbarrier wait is bounded; on expiry the kernel records
 // kErrTimeout in the device error word, all roles leave their loops, the
@@ -71,7 +72,9 @@ struct KCfg {
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kQTile;
   static constexpr int kBiasOff = kKVOff + kStages * kKVTile;  // float [2 slot][2 buf][BN]
-  static constexpr int kItemOff = kBiasOff + 2 * 2 * BN * 4;
+  static constexpr int kEpiOff = kBiasOff + 2 * 2 * BN * 4;     // O staging: 2 KB per softmax warp
+  static constexpr int kEpiWarpBytes = 32 * 32 * 2;             // 32 rows x 32 bf16 columns
+  static constexpr int kItemOff = kEpiOff + 8 * kEpiWarpBytes;
   static constexpr int kBarOff = kItemOff + ((2 * (int)sizeof(Item) + 15) / 16) * 16;
   // barriers: q_full[2] q_empty[2] s_full[2] p_full[2][2 halves] o_full[2]
   //           o_empty[2] item_full[2] item_empty[2] bias_full[2][2] drain
@@ -153,6 +156,7 @@ struct Smem {
   __device__ float* bias(int s, int b) const {
     return reinterpret_cast<float*>(base + KCfg<D>::kBiasOff) + (s * 2 + b) * BN;
   }
+  __device__ uint8_t* epi(int warp) const { return base + KCfg<D>::kEpiOff + warp * KCfg<D>::kEpiWarpBytes; }
   __device__ Item* items() const { return reinterpret_cast<Item*>(base + KCfg<D>::kItemOff); }
   __device__ uint64_t* bars() const { return reinterpret_cast<uint64_t*>(base + KCfg<D>::kBarOff); }
   __device__ uint64_t* q_full(int s) const { return bars() + 0 + s; }
@@ -624,8 +628,17 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
       ptx::tc_fence_after();
     }
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) +
-                          ((long long)(q_row0 + r) * p.n_heads + head) * D;
+    // O / l -> bf16, 32 columns at a time, through a 2 KB per-warp staging
+    // block so that the global stores are coalesced: each thread writes its
+    // row's 64 bytes into the block, then every store instruction of the warp
+    // writes 8 rows x 64 contiguous bytes (4 lanes per row) instead of 32
+    // scattered 16-byte pieces. The block holds 32 rows x 4 16-byte units;
+    // unit c of row x sits at 4x + (c ^ ((x >> 1) & 3)), which keeps both the
+    // row-wise writes and the 8-row reads free of bank conflicts.
+    const int lane = threadIdx.x & 31;
+    const uint32_t stg = ptx::smem_u32(sm.epi(warp));
+    auto unit_addr = [&](int x, int c) { return stg + (uint32_t)(4 * x + (c ^ ((x >> 1) & 3))) * 16u; };
+    const int wrow0 = (warp & 3) * 32;  // first tile row of this warp
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
       uint32_t o[32];
@@ -636,15 +649,24 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[e] = 0u;
       }
-      if (row_ok) {
-        uint4 v[4];
-        uint32_t* vw = reinterpret_cast<uint32_t*>(v);
+      uint32_t vw[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          vw[e] = ptx::pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+      for (int e = 0; e < 16; ++e)
+        vw[e] = ptx::pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+      __syncwarp();  // the previous block's reads are done
 #pragma unroll
-        for (int e = 0; e < 4; ++e) dst[e] = v[e];
+      for (int u4 = 0; u4 < 4; ++u4)
+        ptx::st_shared_v4(unit_addr(lane, u4), vw[4 * u4], vw[4 * u4 + 1], vw[4 * u4 + 2], vw[4 * u4 + 3]);
+      __syncwarp();
+#pragma unroll
+      for (int k8 = 0; k8 < 4; ++k8) {
+        const int x = 8 * k8 + (lane >> 2), cu = lane & 3;
+        const uint4 val = ptx::ld_shared_v4(unit_addr(x, cu));
+        if (wrow0 + x < rows) {
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) +
+                               ((long long)(q_row0 + wrow0 + x) * p.n_heads + head) * D + c * 32 + cu * 8;
+          *reinterpret_cast<uint4*>(dst) = val;
+        }
       }
     }
     if (n > 0) {
