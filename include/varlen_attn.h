@@ -119,6 +119,33 @@ int varlen_attn_fwd(const void* q, const void* k, const void* v,
                     int64_t bias_stride_q, int64_t bias_stride_k,
                     void* out, float* lse, void* stream);
 
+/* Flags of varlen_attn_fwd_ex. */
+enum {
+  /* The per-pair grid is per K/V head: query head h reads grid head h / G,
+   * i.e. element i*bias_stride_b + (h / G)*bias_stride_h + r*bias_stride_q +
+   * c*bias_stride_k. This is the attention_bias layout (batch, n_kv_heads,
+   * q_len, k_len) of "Flash Dynamic Mask Attention (FDMA) Into
+   * Transformers-Style Attention", Key Implementation Points, Attn Bias Path,
+   * read without expanding it to the query heads. */
+  VARLEN_ATTN_BIAS_PAIR_KV_HEADS = 1
+};
+
+/*
+ * varlen_attn_fwd with option flags (a bitwise OR of the enum above; 0 gives
+ * exactly varlen_attn_fwd). Unknown flag bits return VARLEN_ATTN_ERR_BAD_BIAS.
+ * Same arguments, outputs, ownership and error rules as varlen_attn_fwd.
+ */
+int varlen_attn_fwd_ex(const void* q, const void* k, const void* v,
+                       const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                       int batch, int total_q, int total_k,
+                       int max_seqlen_q, int max_seqlen_k,
+                       int n_heads, int n_kv_heads, int head_dim,
+                       float softmax_scale, int causal,
+                       const float* bias_per_key,
+                       const float* bias_pair, int64_t bias_stride_b, int64_t bias_stride_h,
+                       int64_t bias_stride_q, int64_t bias_stride_k, unsigned flags,
+                       void* out, float* lse, void* stream);
+
 /*
  * Same operation with fp32 q/k/v/out (fp32 arithmetic on the CUDA cores).
  * Same arguments and rules as varlen_attn_fwd, except that q, k, v and out
@@ -174,6 +201,72 @@ int varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                             const float* bias_pair, int64_t bias_stride_b, int64_t bias_stride_h,
                             int64_t bias_stride_q, int64_t bias_stride_k,
                             void* out, float* lse, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Packed-layout helpers (device-side, asynchronous on `stream`).
+ *
+ * They turn a padded batch into the packed stream the forward reads and back
+ * again, following the varlen unpad / pad pipeline of "Flash Dynamic Mask
+ * Attention (FDMA) Into Transformers-Style Attention" (Key Implementation
+ * Points, Variable Length Flow), and fold a per-pair bias row into a per-key
+ * bias ("[GiGL] pull request 858", Approach: with query_is_first_token, row 0
+ * of the per-pair bias is added to the per-key bias). Boundaries and indices
+ * read from device memory are bounds-checked: a bad value raises
+ * VARLEN_ATTN_ERR_BAD_SEQLENS in the device error word and the affected row is
+ * skipped (never read or written out of range).
+ * ------------------------------------------------------------------------ */
+
+/*
+ * Unpadding: mask [batch, seqlen] uint8 (nonzero = valid position), row-major.
+ * Writes cu_seqlens [batch + 1] (sequence b = the valid positions of row b,
+ * in increasing order), indices [cu_seqlens[batch]] (flat padded position
+ * b * seqlen + s of every packed row; capacity batch * seqlen) and
+ * max_seqlen [1] (the largest row count), all int32 device arrays. Three
+ * kernel launches; nothing is read back to the host.
+ */
+int varlen_mask_to_seqlens(const uint8_t* mask, int batch, int seqlen, int32_t* cu_seqlens,
+                           int32_t* indices, int32_t* max_seqlen, void* stream);
+
+/*
+ * Gather (unpad): dst[t] = src[indices[t]] for t < cu_seqlens[batch], rows of
+ * row_bytes bytes (a multiple of 16; src and dst 16-byte aligned). src holds
+ * src_rows rows, dst dst_rows rows, indices at least dst_rows entries.
+ * cu_seqlens[batch] > dst_rows or an index outside [0, src_rows) is a device
+ * error (VARLEN_ATTN_ERR_BAD_SEQLENS). Rows of dst past cu_seqlens[batch] are
+ * not written.
+ */
+int varlen_gather_rows(const void* src, int64_t src_rows, int64_t row_bytes,
+                       const int32_t* indices, const int32_t* cu_seqlens, int batch, void* dst,
+                       int64_t dst_rows, void* stream);
+
+/*
+ * Scatter (pad): dst (dst_rows rows of row_bytes bytes) is zeroed, then
+ * dst[indices[t]] = src[t] for t < cu_seqlens[batch]. src holds src_rows rows,
+ * indices at least src_rows entries. cu_seqlens[batch] > src_rows or an index
+ * outside [0, dst_rows) is a device error. Same alignment rules as the gather.
+ */
+int varlen_scatter_rows(const void* src, int64_t src_rows, int64_t row_bytes,
+                        const int32_t* indices, const int32_t* cu_seqlens, int batch, void* dst,
+                        int64_t dst_rows, void* stream);
+
+/*
+ * First-token fold: for every sequence i and key c < Lk_i (Lk_i from
+ * cu_seqlens_k) and head h < n_heads,
+ *   bias_out[cu_k[i] + c, h] = (bias_in ? bias_in[cu_k[i] + c, h] : 0)
+ *       + bias_pair[i*bias_stride_b + (h / head_div)*bias_stride_h
+ *                   + row*bias_stride_q + c*bias_stride_k]
+ * with head_div = 1 for a grid over query heads, G for a grid over K/V heads.
+ * bias_in and bias_out are [total_k, n_heads] fp32 (they may be the same
+ * array); key rows past cu_seqlens_k[batch] are not written. A forward whose
+ * sequences each query only row `row` then gives the same result with
+ * bias_out as its per-key bias and no per-pair grid. The caller guarantees
+ * that the grid covers the entries read.
+ */
+int varlen_fold_pair_bias_row(const float* bias_pair, int64_t bias_stride_b,
+                              int64_t bias_stride_h, int64_t bias_stride_q, int64_t bias_stride_k,
+                              int row, int head_div, const int32_t* cu_seqlens_k, int batch,
+                              int total_k, int n_heads, const float* bias_in, float* bias_out,
+                              void* stream);
 
 /* Static description of a status code. Never NULL. */
 const char* varlen_attn_strerror(int status);

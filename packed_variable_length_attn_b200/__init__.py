@@ -22,13 +22,16 @@ import os
 from typing import Optional, Sequence, Tuple
 
 __all__ = ["varlen_attn_fwd", "varlen_attn_fwd_noalloc", "library_path", "load_library", "VarlenAttnError",
-           "get_device_error", "set_profile_events", "launches_per_call", "exported_symbols"]
+           "get_device_error", "set_profile_events", "launches_per_call", "exported_symbols",
+           "mask_to_seqlens", "gather_rows", "scatter_rows", "unpad", "pad", "fold_pair_bias_row",
+           "BIAS_PAIR_KV_HEADS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libvarlen_attn.so")
 _lib = None
 
-# Status codes of include/varlen_attn.h
+# Status codes and flags of include/varlen_attn.h
+BIAS_PAIR_KV_HEADS = 1
 OK = 0
 ERR_BAD_SEQLENS = 9
 ERR_DEVICE_TIMEOUT = 10
@@ -48,7 +51,9 @@ def exported_symbols() -> Tuple[str, ...]:
     return ("varlen_attn_fwd", "varlen_attn_fwd_f32", "varlen_attn_strerror",
             "varlen_attn_get_device_error", "varlen_attn_set_profile_events",
             "varlen_attn_launches_per_call", "varlen_attn_version",
-            "varlen_attn_last_error_detail", "varlen_attn_fwd_noalloc")
+            "varlen_attn_last_error_detail", "varlen_attn_fwd_noalloc", "varlen_attn_fwd_ex",
+            "varlen_mask_to_seqlens", "varlen_gather_rows", "varlen_scatter_rows",
+            "varlen_fold_pair_bias_row")
 
 
 def load_library():
@@ -69,6 +74,17 @@ def load_library():
     lib.varlen_attn_fwd_f32.restype = i32
     lib.varlen_attn_fwd_noalloc.argtypes = fwd_args
     lib.varlen_attn_fwd_noalloc.restype = i32
+    lib.varlen_attn_fwd_ex.argtypes = fwd_args[:21] + [ctypes.c_uint] + fwd_args[21:]
+    lib.varlen_attn_fwd_ex.restype = i32
+    lib.varlen_mask_to_seqlens.argtypes = [vp, i32, i32, vp, vp, vp, vp]
+    lib.varlen_mask_to_seqlens.restype = i32
+    lib.varlen_gather_rows.argtypes = [vp, i64, i64, vp, vp, i32, vp, i64, vp]
+    lib.varlen_gather_rows.restype = i32
+    lib.varlen_scatter_rows.argtypes = [vp, i64, i64, vp, vp, i32, vp, i64, vp]
+    lib.varlen_scatter_rows.restype = i32
+    lib.varlen_fold_pair_bias_row.argtypes = [vp, i64, i64, i64, i64, i32, i32, vp, i32, i32,
+                                              i32, vp, vp, vp]
+    lib.varlen_fold_pair_bias_row.restype = i32
     lib.varlen_attn_strerror.argtypes = [i32]
     lib.varlen_attn_strerror.restype = ctypes.c_char_p
     lib.varlen_attn_get_device_error.argtypes = [vp]
@@ -141,14 +157,17 @@ def _grid_strides(bias_pair, bias_pair_strides: Optional[Sequence[int]]):
 def varlen_attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
                     softmax_scale: Optional[float] = None, causal: bool = False,
                     bias_per_key=None, bias_pair=None, bias_pair_strides=None,
-                    out=None, lse=None, return_lse: bool = True, stream=None):
+                    out=None, lse=None, return_lse: bool = True, stream=None,
+                    bias_pair_kv_heads: bool = False):
     """Packed variable-length attention forward through the C ABI.
 
     bf16 q/k/v run the tensor-core kernel; fp32 q/k/v run the fp32 kernel.
     ``bias_per_key``: fp32 ``[total_k, n_heads]``. ``bias_pair``: fp32 grid
     read at ``i*sb + h*sh + r*sq + c*sk``; strides default to the tensor's own
     (a 4-D ``[B, 1 or H, R, C]`` view, permuted views included; a size-1 head
-    axis broadcasts). Returns ``(out, lse)`` (``lse`` None if not requested).
+    axis broadcasts). ``bias_pair_kv_heads``: the grid is per K/V head
+    (``[B, n_kv_heads, R, C]``; query head h reads grid head h // G; bf16 only).
+    Returns ``(out, lse)`` (``lse`` None if not requested).
     """
     import torch
     lib = load_library()
@@ -196,13 +215,20 @@ def varlen_attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_
     elif lse is not None and (lse.shape != (n_heads, total_q) or lse.dtype != torch.float32
                               or not lse.is_contiguous()):
         raise ValueError("lse must be contiguous fp32 [n_heads, total_q]")
-    fn = lib.varlen_attn_fwd if q.dtype == torch.bfloat16 else lib.varlen_attn_fwd_f32
     ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    args = (ptr(q), ptr(k), ptr(v), ptr(cu_seqlens_q), ptr(cu_seqlens_k), batch, total_q,
+            total_k, int(max_seqlen_q), int(max_seqlen_k), n_heads, n_kv_heads, head_dim,
+            float(softmax_scale), 1 if causal else 0, ptr(bias_per_key), ptr(bias_pair), *strides)
+    tail = (ptr(out), ptr(lse), _stream_handle(stream))
     with torch.cuda.device(dev):
-        status = fn(ptr(q), ptr(k), ptr(v), ptr(cu_seqlens_q), ptr(cu_seqlens_k), batch,
-                    total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), n_heads, n_kv_heads,
-                    head_dim, float(softmax_scale), 1 if causal else 0, ptr(bias_per_key),
-                    ptr(bias_pair), *strides, ptr(out), ptr(lse), _stream_handle(stream))
+        if bias_pair_kv_heads:
+            if q.dtype != torch.bfloat16:
+                raise ValueError("bias_pair_kv_heads is a bf16-path option")
+            status = lib.varlen_attn_fwd_ex(*args, BIAS_PAIR_KV_HEADS, *tail)
+        elif q.dtype == torch.bfloat16:
+            status = lib.varlen_attn_fwd(*args, *tail)
+        else:
+            status = lib.varlen_attn_fwd_f32(*args, *tail)
     _check(status)
     return out, lse
 
@@ -247,3 +273,107 @@ def varlen_attn_fwd_noalloc(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: i
             *strides, ptr(out), ptr(lse), _stream_handle(stream))
     _check(status)
     return out, lse
+
+
+# ----------------------------------------------------------------------------- layout helpers
+
+def _dev_ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def mask_to_seqlens(mask, stream=None):
+    """Unpadding metadata from a [batch, seqlen] validity mask (bool or uint8,
+    CUDA, contiguous): ``(cu_seqlens [B+1], indices [B*S], max_seqlen [1])``,
+    int32 device tensors; the first ``cu_seqlens[-1]`` indices are the flat
+    padded positions of the packed rows. Nothing is read back to the host."""
+    import torch
+    if mask.dim() != 2 or mask.device.type != "cuda":
+        raise ValueError("mask must be a 2-D CUDA tensor [batch, seqlen]")
+    m = mask.to(torch.uint8).contiguous()
+    B, S = m.shape
+    cu = torch.empty(B + 1, dtype=torch.int32, device=m.device)
+    idx = torch.empty(B * S, dtype=torch.int32, device=m.device)
+    mx = torch.empty(1, dtype=torch.int32, device=m.device)
+    with torch.cuda.device(m.device):
+        _check(load_library().varlen_mask_to_seqlens(_dev_ptr(m), B, S, _dev_ptr(cu),
+                                                     _dev_ptr(idx), _dev_ptr(mx),
+                                                     _stream_handle(stream)))
+    return cu, idx, mx
+
+
+def _rows_view(t):
+    if not t.is_contiguous() or t.dim() < 1:
+        raise ValueError("row tensors must be contiguous")
+    row_bytes = t.element_size() * (t.numel() // max(1, t.shape[0])) if t.shape[0] else 0
+    return t.shape[0], row_bytes
+
+
+def gather_rows(src, indices, cu_seqlens, out, stream=None):
+    """out[t] = src[indices[t]] for t < cu_seqlens[-1] (rows = first dimension;
+    row size a multiple of 16 bytes)."""
+    import torch
+    n_src, rb = _rows_view(src)
+    n_dst, rb2 = _rows_view(out)
+    if rb != rb2 or src.dtype != out.dtype:
+        raise ValueError("src and out rows must match in size and dtype")
+    with torch.cuda.device(src.device):
+        _check(load_library().varlen_gather_rows(
+            _dev_ptr(src), n_src, rb, _dev_ptr(indices), _dev_ptr(cu_seqlens),
+            cu_seqlens.numel() - 1, _dev_ptr(out), n_dst, _stream_handle(stream)))
+    return out
+
+
+def scatter_rows(src, indices, cu_seqlens, out, stream=None):
+    """out = 0, then out[indices[t]] = src[t] for t < cu_seqlens[-1]."""
+    import torch
+    n_src, rb = _rows_view(src)
+    n_dst, rb2 = _rows_view(out)
+    if rb != rb2 or src.dtype != out.dtype:
+        raise ValueError("src and out rows must match in size and dtype")
+    with torch.cuda.device(src.device):
+        _check(load_library().varlen_scatter_rows(
+            _dev_ptr(src), n_src, rb, _dev_ptr(indices), _dev_ptr(cu_seqlens),
+            cu_seqlens.numel() - 1, _dev_ptr(out), n_dst, _stream_handle(stream)))
+    return out
+
+
+def unpad(x, mask, stream=None):
+    """Padded ``x [B, S, ...]`` + mask ``[B, S]`` -> ``(packed [T, ...], indices,
+    cu_seqlens, max_seqlen)``. Sizing the packed tensor reads T back to the host
+    (one synchronisation), as the padded-to-packed conversion of the
+    FlashAttention pipeline does."""
+    import torch
+    B, S = mask.shape
+    cu, idx, mx = mask_to_seqlens(mask, stream)
+    T = int(cu[-1].item())
+    packed = torch.empty((T,) + tuple(x.shape[2:]), dtype=x.dtype, device=x.device)
+    if T:
+        gather_rows(x.reshape((B * S,) + tuple(x.shape[2:])), idx, cu, packed, stream)
+    return packed, idx[:T], cu, int(mx.item())
+
+
+def pad(packed, indices, cu_seqlens, batch, seqlen, stream=None):
+    """Packed ``[T, ...]`` -> padded ``[batch, seqlen, ...]`` (zeros elsewhere)."""
+    import torch
+    out = torch.empty((batch * seqlen,) + tuple(packed.shape[1:]), dtype=packed.dtype,
+                      device=packed.device)
+    scatter_rows(packed, indices, cu_seqlens, out, stream)
+    return out.reshape((batch, seqlen) + tuple(packed.shape[1:]))
+
+
+def fold_pair_bias_row(bias_pair, cu_seqlens_k, n_heads, total_k, row=0, head_div=1,
+                       bias_pair_strides=None, bias_in=None, out=None, stream=None):
+    """Per-key bias ``[total_k, n_heads]`` = ``bias_in`` (or 0) + row ``row`` of
+    the per-pair grid (first-token fold; ``head_div`` = G for a grid over K/V
+    heads)."""
+    import torch
+    strides = _grid_strides(bias_pair, bias_pair_strides)
+    if out is None:
+        out = torch.empty((total_k, n_heads), dtype=torch.float32, device=bias_pair.device)
+    with torch.cuda.device(bias_pair.device):
+        _check(load_library().varlen_fold_pair_bias_row(
+            _dev_ptr(bias_pair), *strides, int(row), int(head_div), _dev_ptr(cu_seqlens_k),
+            cu_seqlens_k.numel() - 1, int(total_k), int(n_heads),
+            None if bias_in is None else _dev_ptr(bias_in), _dev_ptr(out),
+            _stream_handle(stream)))
+    return out

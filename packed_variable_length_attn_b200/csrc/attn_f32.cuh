@@ -30,6 +30,7 @@ struct F32Params {
   const float* bias_key;
   const float* bias_pair;
   long long sb, sh, sr, sc;
+  int bias_head_div;  // grid head index = head / bias_head_div
   float* out;
   float* lse;
   const int* valid;  // work count written by the validation pass (0 = invalid input)
@@ -88,7 +89,8 @@ __global__ void __launch_bounds__(kF32Threads) attn_fwd_f32(const F32Params p) {
   for (int t = 0; t < D / 4; ++t) acc[t] = 0.f;
   const float* brow = nullptr;
   if (p.bias_pair != nullptr && row_ok)
-    brow = p.bias_pair + (long long)i * p.sb + (long long)h * p.sh + (long long)q_loc * p.sr;
+    brow = p.bias_pair + (long long)i * p.sb + (long long)(h / p.bias_head_div) * p.sh +
+           (long long)q_loc * p.sr;
 
   for (int kt = 0; kt < ntiles; ++kt) {
     const int kb = kt * kF32Keys;

@@ -486,7 +486,7 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
     const int limit = p.causal ? min(Lk, q_loc + (Lk - Lq) + 1) : Lk;
     const float* brow = nullptr;
     if (kBiasPair && row_ok)
-      brow = p.bias_pair + (long long)seq * p.sb + (long long)head * p.sh +
+      brow = p.bias_pair + (long long)seq * p.sb + (long long)(head / p.bias_head_div) * p.sh +
              (long long)q_loc * p.sr;
     float m_used = -INFINITY, l = 0.f;
 

@@ -50,6 +50,8 @@ struct AttnParams {
   const float* bias_key;           // [Tk, Hq] or null
   const float* bias_pair;          // strided grid or null
   long long sb, sh, sr, sc;
+  int bias_head_div;               // grid head index = head / bias_head_div (1: query
+                                   // heads; G: K/V heads)
   int pair_vec;                    // 1: 16-byte vector loads of the grid are legal
   void* out;                       // bf16 [Tq, Hq, D]
   float* lse;                      // [Hq, Tq] or null

@@ -9,6 +9,7 @@
 #include <cstdio>
 #include <cstring>
 #include <map>
+#include <algorithm>
 #include <mutex>
 #include <utility>
 
@@ -16,6 +17,7 @@
 #include "attn_f32.cuh"
 #include "attn_sm100.cuh"
 #include "sched.cuh"
+#include "layout.cuh"
 
 // ---------------------------------------------------------------------------
 // Fixed scratch for varlen_attn_fwd_noalloc.
@@ -260,17 +262,13 @@ int noalloc_scratch(void** out) {
   return VARLEN_ATTN_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-int varlen_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
-                    const int32_t* cu_seqlens_k, int batch, int total_q, int total_k,
-                    int max_seqlen_q, int max_seqlen_k, int n_heads, int n_kv_heads, int head_dim,
-                    float softmax_scale, int causal, const float* bias_per_key,
-                    const float* bias_pair, int64_t bias_stride_b, int64_t bias_stride_h,
-                    int64_t bias_stride_q, int64_t bias_stride_k, void* out, float* lse,
-                    void* stream) {
+int fwd_bf16(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+             const int32_t* cu_seqlens_k, int batch, int total_q, int total_k, int max_seqlen_q,
+             int max_seqlen_k, int n_heads, int n_kv_heads, int head_dim, float softmax_scale,
+             int causal, const float* bias_per_key, const float* bias_pair, int64_t bias_stride_b,
+             int64_t bias_stride_h, int64_t bias_stride_q, int64_t bias_stride_k, unsigned flags,
+             void* out, float* lse, void* stream) {
+  if (flags & ~(unsigned)VARLEN_ATTN_BIAS_PAIR_KV_HEADS) return VARLEN_ATTN_ERR_BAD_BIAS;
   Common a{batch, total_q, total_k, max_seqlen_q, max_seqlen_k, n_heads, n_kv_heads, head_dim,
            causal ? 1 : 0, cu_seqlens_q, cu_seqlens_k, bias_per_key, bias_pair, bias_stride_b,
            bias_stride_h, bias_stride_q, bias_stride_k};
@@ -330,6 +328,7 @@ int varlen_attn_fwd(const void* q, const void* k, const void* v, const int32_t* 
   prm.bias_pair = bias_pair;
   prm.sb = bias_stride_b;
   prm.sh = bias_stride_h;
+  prm.bias_head_div = (flags & VARLEN_ATTN_BIAS_PAIR_KV_HEADS) ? G : 1;
   prm.sr = bias_stride_q;
   prm.sc = bias_stride_k;
   prm.pair_vec = bias_pair && bias_stride_k == 1 && aligned(bias_pair, 16) &&
@@ -363,6 +362,52 @@ int varlen_attn_fwd(const void* q, const void* k, const void* v, const int32_t* 
     if (e != cudaSuccess) return cuda_fail("cudaEventRecord(stop)", e);
   }
   return VARLEN_ATTN_OK;
+}
+
+int layout_grid(const DeviceInfo* di, int64_t units) {
+  const int64_t want = (units + kLayoutThreads - 1) / kLayoutThreads;
+  const int64_t cap = (int64_t)di->sm_count * 8;
+  return (int)std::max<int64_t>(1, std::min(want, cap));
+}
+
+int rows_args_ok(const void* src, int64_t src_rows, int64_t row_bytes, const int32_t* indices,
+                 const int32_t* cu, int batch, const void* dst, int64_t dst_rows) {
+  if (!src || !dst || !indices || !cu) return VARLEN_ATTN_ERR_NULL_POINTER;
+  if (batch <= 0 || src_rows < 0 || dst_rows < 0 || row_bytes <= 0 || row_bytes % 16 != 0)
+    return VARLEN_ATTN_ERR_BAD_SHAPE;
+  if (!aligned(src, 16) || !aligned(dst, 16) || !aligned(indices, 4) || !aligned(cu, 4))
+    return VARLEN_ATTN_ERR_MISALIGNED;
+  return VARLEN_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int varlen_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                    const int32_t* cu_seqlens_k, int batch, int total_q, int total_k,
+                    int max_seqlen_q, int max_seqlen_k, int n_heads, int n_kv_heads, int head_dim,
+                    float softmax_scale, int causal, const float* bias_per_key,
+                    const float* bias_pair, int64_t bias_stride_b, int64_t bias_stride_h,
+                    int64_t bias_stride_q, int64_t bias_stride_k, void* out, float* lse,
+                    void* stream) {
+  return fwd_bf16(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+                  max_seqlen_k, n_heads, n_kv_heads, head_dim, softmax_scale, causal, bias_per_key,
+                  bias_pair, bias_stride_b, bias_stride_h, bias_stride_q, bias_stride_k, 0u, out,
+                  lse, stream);
+}
+
+int varlen_attn_fwd_ex(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                       const int32_t* cu_seqlens_k, int batch, int total_q, int total_k,
+                       int max_seqlen_q, int max_seqlen_k, int n_heads, int n_kv_heads,
+                       int head_dim, float softmax_scale, int causal, const float* bias_per_key,
+                       const float* bias_pair, int64_t bias_stride_b, int64_t bias_stride_h,
+                       int64_t bias_stride_q, int64_t bias_stride_k, unsigned flags, void* out,
+                       float* lse, void* stream) {
+  return fwd_bf16(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+                  max_seqlen_k, n_heads, n_kv_heads, head_dim, softmax_scale, causal, bias_per_key,
+                  bias_pair, bias_stride_b, bias_stride_h, bias_stride_q, bias_stride_k, flags, out,
+                  lse, stream);
 }
 
 int varlen_attn_fwd_f32(const float* q, const float* k, const float* v,
@@ -418,6 +463,7 @@ int varlen_attn_fwd_f32(const float* q, const float* k, const float* v,
   prm.bias_pair = bias_pair;
   prm.sb = bias_stride_b;
   prm.sh = bias_stride_h;
+  prm.bias_head_div = 1;
   prm.sr = bias_stride_q;
   prm.sc = bias_stride_k;
   prm.out = out;
@@ -525,6 +571,7 @@ int varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   prm.bias_pair = bias_pair;
   prm.sb = bias_stride_b;
   prm.sh = bias_stride_h;
+  prm.bias_head_div = 1;
   prm.sr = bias_stride_q;
   prm.sc = bias_stride_k;
   prm.pair_vec = bias_pair && bias_stride_k == 1 && aligned(bias_pair, 16) &&
@@ -569,6 +616,80 @@ const char* varlen_attn_strerror(int status) {
       return "work list exceeds the fixed scratch of varlen_attn_fwd_noalloc";
     default: return "unknown status";
   }
+}
+
+int varlen_mask_to_seqlens(const uint8_t* mask, int batch, int seqlen, int32_t* cu_seqlens,
+                           int32_t* indices, int32_t* max_seqlen, void* stream) {
+  if (!mask || !cu_seqlens || !indices || !max_seqlen) return VARLEN_ATTN_ERR_NULL_POINTER;
+  if (batch <= 0 || seqlen <= 0) return VARLEN_ATTN_ERR_BAD_SHAPE;
+  if ((int64_t)batch * seqlen > INT32_MAX) return VARLEN_ATTN_ERR_TOO_LARGE;
+  if (!aligned(cu_seqlens, 4) || !aligned(indices, 4) || !aligned(max_seqlen, 4))
+    return VARLEN_ATTN_ERR_MISALIGNED;
+  DeviceInfo* di = nullptr;
+  if (int rc = device_info(&di)) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  mask_count_kernel<<<batch, kLayoutThreads, 0, st>>>(mask, seqlen, cu_seqlens + 1);
+  if (int rc = check_launch("launch mask_count_kernel")) return rc;
+  seqlens_scan_kernel<<<1, kLayoutThreads, 0, st>>>(cu_seqlens, batch, max_seqlen);
+  if (int rc = check_launch("launch seqlens_scan_kernel")) return rc;
+  mask_indices_kernel<<<batch, kLayoutThreads, 0, st>>>(mask, seqlen, cu_seqlens, indices);
+  return check_launch("launch mask_indices_kernel");
+}
+
+
+int varlen_gather_rows(const void* src, int64_t src_rows, int64_t row_bytes,
+                       const int32_t* indices, const int32_t* cu_seqlens, int batch, void* dst,
+                       int64_t dst_rows, void* stream) {
+  if (int rc = rows_args_ok(src, src_rows, row_bytes, indices, cu_seqlens, batch, dst, dst_rows))
+    return rc;
+  DeviceInfo* di = nullptr;
+  if (int rc = device_info(&di)) return rc;
+  const int64_t units = row_bytes / 16;
+  gather_rows_kernel<<<layout_grid(di, dst_rows * units), kLayoutThreads, 0,
+                       static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(src), src_rows, units, indices, cu_seqlens, batch,
+      static_cast<uint4*>(dst), dst_rows, di->error_word);
+  return check_launch("launch gather_rows_kernel");
+}
+
+int varlen_scatter_rows(const void* src, int64_t src_rows, int64_t row_bytes,
+                        const int32_t* indices, const int32_t* cu_seqlens, int batch, void* dst,
+                        int64_t dst_rows, void* stream) {
+  if (int rc = rows_args_ok(src, src_rows, row_bytes, indices, cu_seqlens, batch, dst, dst_rows))
+    return rc;
+  DeviceInfo* di = nullptr;
+  if (int rc = device_info(&di)) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(dst, 0, (size_t)(dst_rows * row_bytes), st);
+  if (e != cudaSuccess) return cuda_fail("cudaMemsetAsync(padded rows)", e);
+  const int64_t units = row_bytes / 16;
+  scatter_rows_kernel<<<layout_grid(di, src_rows * units), kLayoutThreads, 0, st>>>(
+      static_cast<const uint4*>(src), src_rows, units, indices, cu_seqlens, batch,
+      static_cast<uint4*>(dst), dst_rows, di->error_word);
+  return check_launch("launch scatter_rows_kernel");
+}
+
+int varlen_fold_pair_bias_row(const float* bias_pair, int64_t bias_stride_b,
+                              int64_t bias_stride_h, int64_t bias_stride_q, int64_t bias_stride_k,
+                              int row, int head_div, const int32_t* cu_seqlens_k, int batch,
+                              int total_k, int n_heads, const float* bias_in, float* bias_out,
+                              void* stream) {
+  if (!bias_pair || !cu_seqlens_k || !bias_out) return VARLEN_ATTN_ERR_NULL_POINTER;
+  if (batch <= 0 || total_k < 0 || n_heads <= 0 || head_div <= 0 || row < 0)
+    return VARLEN_ATTN_ERR_BAD_SHAPE;
+  if (bias_stride_b < 0 || bias_stride_h < 0 || bias_stride_q < 0 || bias_stride_k < 0)
+    return VARLEN_ATTN_ERR_BAD_BIAS;
+  if ((int64_t)total_k * n_heads > INT32_MAX) return VARLEN_ATTN_ERR_TOO_LARGE;
+  if (!aligned(bias_pair, 4) || !aligned(bias_out, 4) || (bias_in && !aligned(bias_in, 4)) ||
+      !aligned(cu_seqlens_k, 4))
+    return VARLEN_ATTN_ERR_MISALIGNED;
+  DeviceInfo* di = nullptr;
+  if (int rc = device_info(&di)) return rc;
+  fold_pair_row_kernel<<<layout_grid(di, (int64_t)total_k * n_heads), kLayoutThreads, 0,
+                         static_cast<cudaStream_t>(stream)>>>(
+      bias_pair, bias_stride_b, bias_stride_h, bias_stride_q, bias_stride_k, row, head_div,
+      cu_seqlens_k, batch, total_k, n_heads, bias_in, bias_out, di->error_word);
+  return check_launch("launch fold_pair_row_kernel");
 }
 
 int varlen_attn_get_device_error(void* stream) {

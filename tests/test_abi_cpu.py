@@ -26,7 +26,7 @@ def _declared():
         if fn.endswith(".h"):
             src = open(os.path.join(ROOT, "include", fn)).read()
             src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-            names += re.findall(r"^\s*(?:const\s+)?\w+\s*\**\s*(varlen_attn_\w+)\s*\(", src, flags=re.M)
+            names += re.findall(r"^\s*(?:const\s+)?\w+\s*\**\s*(varlen_\w+)\s*\(", src, flags=re.M)
     return sorted(set(names))
 
 
@@ -92,3 +92,24 @@ def test_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(va, "_LIB_PATH", "/nonexistent/libvarlen_attn.so")
     with pytest.raises(ImportError):
         va.load_library()
+
+
+def test_helper_host_validation_codes(lib):
+    p = ctypes.c_void_p
+    # varlen_attn_fwd_ex: unknown flag bits are rejected before any device work
+    assert lib.varlen_attn_fwd_ex(p(16), p(16), p(16), p(16), p(16), 1, 8, 8, 8, 8, 2, 2, 64,
+                                  0.125, 1, None, None, 0, 0, 0, 0, 2, p(16), p(16), None) == 6
+    assert lib.varlen_mask_to_seqlens(None, 2, 4, p(16), p(16), p(16), None) == 1
+    assert lib.varlen_mask_to_seqlens(p(16), 0, 4, p(16), p(16), p(16), None) == 2
+    assert lib.varlen_mask_to_seqlens(p(16), 2, 4, p(18), p(16), p(16), None) == 5
+    assert lib.varlen_mask_to_seqlens(p(16), 1 << 16, 1 << 16, p(16), p(16), p(16), None) == 11
+    for fn in (lib.varlen_gather_rows, lib.varlen_scatter_rows):
+        assert fn(None, 4, 32, p(16), p(16), 1, p(16), 4, None) == 1
+        assert fn(p(16), 4, 24, p(16), p(16), 1, p(16), 4, None) == 2   # rows not 16-byte units
+        assert fn(p(16), 4, 32, p(16), p(16), 0, p(16), 4, None) == 2
+        assert fn(p(24), 4, 32, p(16), p(16), 1, p(16), 4, None) == 5
+    f = lib.varlen_fold_pair_bias_row
+    assert f(None, 0, 0, 1, 1, 0, 1, p(16), 1, 4, 2, None, p(16), None) == 1
+    assert f(p(16), 0, 0, 1, 1, 0, 0, p(16), 1, 4, 2, None, p(16), None) == 2   # head_div 0
+    assert f(p(16), 0, -1, 1, 1, 0, 1, p(16), 1, 4, 2, None, p(16), None) == 6
+    assert f(p(16), 0, 0, 1, 1, 0, 1, p(16), 1, 4, 2, p(18), p(16), None) == 5
