@@ -463,6 +463,68 @@ def run_gpu(args, world, rank, local):
         dist.destroy_process_group()
 
 
+def run_layout(args, world, rank, local):
+    """Packed-layout helpers on the long workload's Q padded to [16, 8192, 32, 128]
+    bf16 (1.07 GB): unpad = mask_to_seqlens + gather_rows, pad = scatter_rows
+    (zero fill + scatter). HBM-bound copies, reported as GB/s of the bytes they
+    must move against the measured HBM peak. One JSON line per helper."""
+    import torch
+    import packed_variable_length_attn_b200 as va
+    if rank != 0:
+        return
+    torch.cuda.set_device(local)
+    w = _workload(args, seed=rank_seed(0, WORKLOAD))
+    B, S = w.batch, 8192
+    H, D = w.n_heads, w.head_dim
+    dev = torch.device("cuda", local)
+    mask = torch.zeros(B, S, dtype=torch.uint8, device=dev)
+    for b, L in enumerate(w.lengths_q):
+        mask[b, :L] = 1
+    x = torch.empty(B * S, H, D, dtype=torch.bfloat16, device=dev).normal_()
+    T = w.total_q
+    rb = H * D * 2
+    packed = torch.empty(T, H, D, dtype=torch.bfloat16, device=dev)
+    padded = torch.empty_like(x)
+    peaks, src = _peaks()
+    cu, idx, mx = va.mask_to_seqlens(mask)
+
+    def unpad():
+        c, i, _ = va.mask_to_seqlens(mask)
+        va.gather_rows(x, i, c, packed)
+
+    def pad():
+        va.scatter_rows(packed, idx, cu, padded)
+
+    ops = {"unpad": (unpad, B * S + 2 * T * rb + 4 * (B + 1) + 4 * T),
+           "pad": (pad, B * S * rb + 2 * T * rb)}
+    for name, (fn, nbytes) in ops.items():
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(args.steps):
+            fn()
+        t1.record()
+        torch.cuda.synchronize()
+        ms = t0.elapsed_time(t1) / args.steps
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        if va.get_device_error() != 0:
+            raise RuntimeError("device error in the layout helpers")
+        print(json.dumps({
+            "metric": f"{name} (packed-layout helper) GB/s on 1 B200", "value": gbs,
+            "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": max(3, args.warmup),
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (the long workload's lengths as prefix masks)",
+            "config": {"workload": f"{name}_long_causal_gqa_q", "batch": B, "seqlen": S,
+                       "heads": H, "head_dim": D, "packed_rows": T, "row_bytes": rb},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]),
+                         "unit": "GB/s", "frac": gbs / float(peaks["hbm_gbs"]),
+                         "algorithmic_bytes_per_step": nbytes, "traffic": None,
+                         "peak_source": f"{src} hbm_gbs"}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -479,12 +541,17 @@ def main():
                     help="named workload (default: the long causal GQA workload)")
     ap.add_argument("--flush-l2", action="store_true",
                     help="256 MB scrub write between timed steps; each call timed alone")
+    ap.add_argument("--layout", action="store_true",
+                    help="time the packed-layout helpers (unpad, pad) instead of the forward")
     ap.add_argument("--sequences", type=int, default=0,
                     help="use only the first N sequences (small case for profiling)")
     args = ap.parse_args()
     world, rank, local = _dist()
     if args.impl == "reference":
         run_reference(args, world, rank)
+        return
+    if args.layout:
+        run_layout(args, world, rank, local)
         return
     run_gpu(args, world, rank, local)
 
