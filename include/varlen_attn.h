@@ -202,6 +202,41 @@ int varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                             int64_t bias_stride_q, int64_t bias_stride_k,
                             void* out, float* lse, void* stream);
 
+/*
+ * Decode attention over a per-sequence K/V cache (flash_attn_with_kvcache in
+ * "fix(flex): avoid decoding kernel selection for short GQA" and the noether
+ * attention module page; q_len = 1 decode steps, FDMA integration page,
+ * Causality Handling). Same definition as varlen_attn_fwd with the keys and
+ * values of sequence i taken from the cache:
+ *
+ *   k_cache, v_cache  [batch, cache_len, n_kv_heads, head_dim] bf16; sequence
+ *            i's cached rows are i*cache_len .. i*cache_len + cache_seqlens[i]-1.
+ *   k_new, v_new      NULL (both), or [total_q, n_kv_heads, head_dim] bf16
+ *            packed like q: sequence i's new rows are first written into its
+ *            cache rows cache_seqlens[i] .. cache_seqlens[i] + Lq_i - 1 (the
+ *            cache is modified; cache_seqlens is not), and attended to.
+ *   Lk_i = cache_seqlens[i] (+ Lq_i with new rows); causal is bottom-right as
+ *   in varlen_attn_fwd (with Lq_i = 1 it changes nothing).
+ *   q [total_q, n_heads, head_dim] bf16 with cu_seqlens_q [batch + 1];
+ *   max_seqlen_q * (n_heads / n_kv_heads) <= 32 (decode-sized queries; longer
+ *   ones belong to varlen_attn_fwd): else VARLEN_ATTN_ERR_BAD_SHAPE.
+ *   out [total_q, n_heads, head_dim] bf16, lse [n_heads, total_q] fp32 or NULL.
+ *   num_splits: key splits per (sequence, K/V head); 0 = chosen from the batch
+ *            size and cache_len. With more than one split, partial results go
+ *            to the library workspace and a third launch merges them; results
+ *            depend on the split count in the last bits (the merge order), so
+ *            give a fixed num_splits where bitwise reproducibility across batch
+ *            compositions matters.
+ * HBM-bound (every cached key and value is read once): fp32 on the CUDA
+ * cores, no bias. Errors as for varlen_attn_fwd; a cache position beyond
+ * cache_len raises VARLEN_ATTN_ERR_BAD_SEQLENS on the device.
+ */
+int varlen_attn_decode(const void* q, const int32_t* cu_seqlens_q, int batch, int total_q,
+                       int max_seqlen_q, void* k_cache, void* v_cache, int cache_len,
+                       const int32_t* cache_seqlens, const void* k_new, const void* v_new,
+                       int n_heads, int n_kv_heads, int head_dim, float softmax_scale,
+                       int causal, int num_splits, void* out, float* lse, void* stream);
+
 /* ------------------------------------------------------------------------
  * Packed-layout helpers (device-side, asynchronous on `stream`).
  *

@@ -24,7 +24,7 @@ from typing import Optional, Sequence, Tuple
 __all__ = ["varlen_attn_fwd", "varlen_attn_fwd_noalloc", "library_path", "load_library", "VarlenAttnError",
            "get_device_error", "set_profile_events", "launches_per_call", "exported_symbols",
            "mask_to_seqlens", "gather_rows", "scatter_rows", "unpad", "pad", "fold_pair_bias_row",
-           "BIAS_PAIR_KV_HEADS"]
+           "varlen_attn_decode", "BIAS_PAIR_KV_HEADS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libvarlen_attn.so")
@@ -53,7 +53,7 @@ def exported_symbols() -> Tuple[str, ...]:
             "varlen_attn_launches_per_call", "varlen_attn_version",
             "varlen_attn_last_error_detail", "varlen_attn_fwd_noalloc", "varlen_attn_fwd_ex",
             "varlen_mask_to_seqlens", "varlen_gather_rows", "varlen_scatter_rows",
-            "varlen_fold_pair_bias_row")
+            "varlen_fold_pair_bias_row", "varlen_attn_decode")
 
 
 def load_library():
@@ -85,6 +85,9 @@ def load_library():
     lib.varlen_fold_pair_bias_row.argtypes = [vp, i64, i64, i64, i64, i32, i32, vp, i32, i32,
                                               i32, vp, vp, vp]
     lib.varlen_fold_pair_bias_row.restype = i32
+    lib.varlen_attn_decode.argtypes = [vp, vp, i32, i32, i32, vp, vp, i32, vp, vp, vp, i32, i32,
+                                       i32, f32, i32, i32, vp, vp, vp]
+    lib.varlen_attn_decode.restype = i32
     lib.varlen_attn_strerror.argtypes = [i32]
     lib.varlen_attn_strerror.restype = ctypes.c_char_p
     lib.varlen_attn_get_device_error.argtypes = [vp]
@@ -377,3 +380,41 @@ def fold_pair_bias_row(bias_pair, cu_seqlens_k, n_heads, total_k, row=0, head_di
             None if bias_in is None else _dev_ptr(bias_in), _dev_ptr(out),
             _stream_handle(stream)))
     return out
+
+
+def varlen_attn_decode(q, cu_seqlens_q, max_seqlen_q: int, k_cache, v_cache, cache_seqlens,
+                       k_new=None, v_new=None, softmax_scale: Optional[float] = None,
+                       causal: bool = True, num_splits: int = 0, out=None, lse=None,
+                       return_lse: bool = True, stream=None):
+    """Decode attention over a K/V cache ``[batch, cache_len, n_kv_heads, D]``
+    (bf16). ``k_new``/``v_new`` ``[total_q, n_kv_heads, D]`` are written into
+    the cache after ``cache_seqlens[i]`` rows and attended to. Returns
+    ``(out, lse)``."""
+    import torch
+    lib = load_library()
+    if q.dtype != torch.bfloat16 or k_cache.dtype != q.dtype or v_cache.dtype != q.dtype:
+        raise ValueError("q and the cache must be bf16")
+    if k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache and v_cache must be [batch, cache_len, n_kv_heads, head_dim]")
+    for t in (q, k_cache, v_cache, cu_seqlens_q, cache_seqlens):
+        if not t.is_contiguous() or t.device != q.device:
+            raise ValueError("all tensors must be contiguous and on q's device")
+    total_q, n_heads, head_dim = q.shape
+    batch, cache_len, n_kv_heads, dk = k_cache.shape
+    if dk != head_dim or cu_seqlens_q.numel() != batch + 1 or cache_seqlens.numel() != batch:
+        raise ValueError("shapes of q, the cache, cu_seqlens_q and cache_seqlens disagree")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(head_dim)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((n_heads, total_q), dtype=torch.float32, device=q.device)
+    ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    with torch.cuda.device(q.device):
+        status = lib.varlen_attn_decode(
+            ptr(q), ptr(cu_seqlens_q), batch, total_q, int(max_seqlen_q), ptr(k_cache),
+            ptr(v_cache), cache_len, ptr(cache_seqlens), ptr(k_new), ptr(v_new), n_heads,
+            n_kv_heads, head_dim, float(softmax_scale), 1 if causal else 0, int(num_splits),
+            ptr(out), ptr(lse), _stream_handle(stream))
+    _check(status)
+    return out, lse

@@ -18,6 +18,7 @@
 #include "attn_sm100.cuh"
 #include "sched.cuh"
 #include "layout.cuh"
+#include "decode.cuh"
 
 // ---------------------------------------------------------------------------
 // Fixed scratch for varlen_attn_fwd_noalloc.
@@ -690,6 +691,98 @@ int varlen_fold_pair_bias_row(const float* bias_pair, int64_t bias_stride_b,
       bias_pair, bias_stride_b, bias_stride_h, bias_stride_q, bias_stride_k, row, head_div,
       cu_seqlens_k, batch, total_k, n_heads, bias_in, bias_out, di->error_word);
   return check_launch("launch fold_pair_row_kernel");
+}
+
+int varlen_attn_decode(const void* q, const int32_t* cu_seqlens_q, int batch, int total_q,
+                       int max_seqlen_q, void* k_cache, void* v_cache, int cache_len,
+                       const int32_t* cache_seqlens, const void* k_new, const void* v_new,
+                       int n_heads, int n_kv_heads, int head_dim, float softmax_scale,
+                       int causal, int num_splits, void* out, float* lse, void* stream) {
+  if (!q || !cu_seqlens_q || !k_cache || !v_cache || !cache_seqlens || !out)
+    return VARLEN_ATTN_ERR_NULL_POINTER;
+  if ((k_new == nullptr) != (v_new == nullptr)) return VARLEN_ATTN_ERR_NULL_POINTER;
+  if (batch <= 0 || batch > 65535 || total_q < 0 || max_seqlen_q < 0 || cache_len <= 0 ||
+      n_heads <= 0 || n_kv_heads <= 0 || num_splits < 0 || num_splits > 256)
+    return VARLEN_ATTN_ERR_BAD_SHAPE;
+  if (n_heads % n_kv_heads != 0) return VARLEN_ATTN_ERR_GQA_MISMATCH;
+  if (head_dim != 64 && head_dim != 128) return VARLEN_ATTN_ERR_HEAD_DIM;
+  const int G = n_heads / n_kv_heads;
+  if ((int64_t)max_seqlen_q * G > kDecMaxRows) return VARLEN_ATTN_ERR_BAD_SHAPE;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+      (k_new && (!aligned(k_new, 16) || !aligned(v_new, 16))) || (lse && !aligned(lse, 4)) ||
+      !aligned(cu_seqlens_q, 4) || !aligned(cache_seqlens, 4))
+    return VARLEN_ATTN_ERR_MISALIGNED;
+  if ((int64_t)total_q * n_heads * head_dim > INT32_MAX ||
+      (int64_t)batch * cache_len * n_kv_heads * head_dim / 8 > INT32_MAX)
+    return VARLEN_ATTN_ERR_TOO_LARGE;
+  DeviceInfo* di = nullptr;
+  if (int rc = device_info(&di)) return rc;
+  if (total_q == 0 || max_seqlen_q == 0) return VARLEN_ATTN_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // splits: enough CTAs for two per SM, each split at least 256 keys
+  int splits = num_splits;
+  const int max_blocks = (cache_len + kDecKeys - 1) / kDecKeys;
+  if (splits == 0) {
+    const int64_t ctas = (int64_t)batch * n_kv_heads;
+    const int64_t want = (2 * (int64_t)di->sm_count + ctas - 1) / ctas;
+    splits = (int)std::max<int64_t>(1, std::min<int64_t>(want, std::max(1, max_blocks / 4)));
+  }
+  splits = std::min(splits, std::max(1, max_blocks));
+  DecodeParams dp;
+  dp.q = static_cast<const __nv_bfloat16*>(q);
+  dp.cu_q = cu_seqlens_q;
+  dp.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  dp.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  dp.cache_seqlens = cache_seqlens;
+  dp.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  dp.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  dp.batch = batch;
+  dp.total_q = total_q;
+  dp.cache_len = cache_len;
+  dp.n_heads = n_heads;
+  dp.n_kv_heads = n_kv_heads;
+  dp.group = G;
+  dp.causal = causal ? 1 : 0;
+  dp.n_splits = splits;
+  dp.scale_log2 = softmax_scale * 1.4426950408889634f;
+  dp.out = static_cast<__nv_bfloat16*>(out);
+  dp.lse = lse;
+  dp.part_o = nullptr;
+  dp.part_lse = nullptr;
+  dp.error = di->error_word;
+  if (splits > 1) {
+    const size_t po = (size_t)splits * total_q * n_heads * head_dim * sizeof(float);
+    const size_t pl = (size_t)splits * n_heads * total_q * sizeof(float);
+    void* wsp = nullptr;
+    if (int rc = workspace(stream, po + pl, &wsp)) return rc;
+    dp.part_o = static_cast<float*>(wsp);
+    dp.part_lse = reinterpret_cast<float*>(static_cast<char*>(wsp) + po);
+  }
+  const dim3 grid(splits, n_kv_heads, batch);
+  const int rows = (int)std::min<int64_t>((int64_t)total_q * n_heads / (kDecThreads / 32) + 1,
+                                          (int64_t)di->sm_count * 16);
+  if (head_dim == 64) {
+    if (k_new) {
+      decode_append_kernel<64><<<layout_grid(di, (int64_t)total_q * n_kv_heads * 8), kDecThreads,
+                                 0, st>>>(dp);
+      if (int rc = check_launch("launch decode_append_kernel")) return rc;
+    }
+    if (int rc = set_smem(decode_kernel<64>, DecSmem<64>::kBytes)) return rc;
+    decode_kernel<64><<<grid, kDecThreads, DecSmem<64>::kBytes, st>>>(dp);
+    if (int rc = check_launch("launch decode_kernel")) return rc;
+    if (splits > 1) decode_combine_kernel<64><<<rows, kDecThreads, 0, st>>>(dp);
+  } else {
+    if (k_new) {
+      decode_append_kernel<128><<<layout_grid(di, (int64_t)total_q * n_kv_heads * 16),
+                                  kDecThreads, 0, st>>>(dp);
+      if (int rc = check_launch("launch decode_append_kernel")) return rc;
+    }
+    if (int rc = set_smem(decode_kernel<128>, DecSmem<128>::kBytes)) return rc;
+    decode_kernel<128><<<grid, kDecThreads, DecSmem<128>::kBytes, st>>>(dp);
+    if (int rc = check_launch("launch decode_kernel")) return rc;
+    if (splits > 1) decode_combine_kernel<128><<<rows, kDecThreads, 0, st>>>(dp);
+  }
+  return check_launch("launch decode_combine_kernel");
 }
 
 int varlen_attn_get_device_error(void* stream) {

@@ -113,3 +113,26 @@ def test_helper_host_validation_codes(lib):
     assert f(p(16), 0, 0, 1, 1, 0, 0, p(16), 1, 4, 2, None, p(16), None) == 2   # head_div 0
     assert f(p(16), 0, -1, 1, 1, 0, 1, p(16), 1, 4, 2, None, p(16), None) == 6
     assert f(p(16), 0, 0, 1, 1, 0, 1, p(16), 1, 4, 2, p(18), p(16), None) == 5
+
+
+def test_decode_host_validation_codes(lib):
+    p = ctypes.c_void_p
+
+    def call(**kw):
+        a = dict(q=16, cu=16, batch=2, tq=2, mq=1, kc=16, vc=16, cl=64, cs=16, kn=None, vn=None,
+                 hq=8, hkv=2, d=128, scale=0.1, causal=1, splits=0, out=16, lse=16)
+        a.update(kw)
+        q_ = lambda x: None if x is None else p(x)
+        return lib.varlen_attn_decode(q_(a["q"]), q_(a["cu"]), a["batch"], a["tq"], a["mq"],
+                                      q_(a["kc"]), q_(a["vc"]), a["cl"], q_(a["cs"]), q_(a["kn"]),
+                                      q_(a["vn"]), a["hq"], a["hkv"], a["d"], a["scale"],
+                                      a["causal"], a["splits"], q_(a["out"]), q_(a["lse"]), None)
+    assert call(q=None) == 1
+    assert call(kn=16) == 1            # k_new without v_new
+    assert call(batch=0) == 2
+    assert call(cl=0) == 2
+    assert call(splits=-1) == 2
+    assert call(hq=6, hkv=4) == 3
+    assert call(d=96) == 4
+    assert call(mq=9, hq=8, hkv=2) == 2   # 9 x G=4 > 32 rows: the packed forward's job
+    assert call(kc=24) == 5

@@ -1,0 +1,111 @@
+"""GPU parity of the K/V-cache decode path (varlen_attn_decode) against the
+attention oracle run on the packed K/V the cache holds after the append."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import packed_variable_length_attn_b200 as va
+from tests.parity import compare
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    va.get_device_error()
+    yield
+    assert va.get_device_error() == 0
+
+
+def _case(seed, lq, cache_lens, cache_len, hq, hkv, d, new):
+    g = torch.Generator().manual_seed(seed)
+    B = len(lq)
+    cu_q = torch.tensor(np.concatenate([[0], np.cumsum(lq)]), dtype=torch.int32)
+    Tq = int(cu_q[-1])
+    q = torch.randn(Tq, hq, d, generator=g).to(torch.bfloat16)
+    kc = torch.randn(B, cache_len, hkv, d, generator=g).to(torch.bfloat16)
+    vc = torch.randn(B, cache_len, hkv, d, generator=g).to(torch.bfloat16)
+    cs = torch.tensor(cache_lens, dtype=torch.int32)
+    kn = torch.randn(Tq, hkv, d, generator=g).to(torch.bfloat16) if new else None
+    vn = torch.randn(Tq, hkv, d, generator=g).to(torch.bfloat16) if new else None
+    return cu_q, q, kc, vc, cs, kn, vn
+
+
+def _expected_cache(kc, cs, cu_q, kn):
+    exp = kc.clone()
+    if kn is not None:
+        for i in range(len(cs)):
+            a, b = int(cu_q[i]), int(cu_q[i + 1])
+            exp[i, int(cs[i]):int(cs[i]) + (b - a)] = kn[a:b]
+    return exp
+
+
+def _oracle(q, cu_q, kcache, vcache, lk, hq, hkv, scale, causal):
+    k = torch.cat([kcache[i, :lk[i]] for i in range(len(lk))])
+    v = torch.cat([vcache[i, :lk[i]] for i in range(len(lk))])
+    cu_k = torch.tensor(np.concatenate([[0], np.cumsum(lk)]), dtype=torch.int32)
+    return oracle.fwd(q, k, v, cu_q, cu_k, hq, hkv, scale, causal)
+
+
+CASES = [
+    # lq, cache lens, cache_len, hq, hkv, d, new rows, splits
+    ([1] * 8, [700, 1, 0, 4096, 129, 64, 2000, 3333], 4096, 32, 8, 128, False, 0),
+    ([1] * 8, [700, 1, 0, 4096, 129, 64, 2000, 3333], 4096, 32, 8, 128, False, 1),
+    ([1] * 5, [10, 300, 511, 0, 77], 512, 16, 4, 64, True, 0),
+    ([4, 1, 8, 2], [100, 0, 300, 1000], 1024, 8, 2, 128, True, 3),
+    ([1] * 3, [5000, 17, 8000], 8192, 14, 2, 64, True, 7),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"B{len(c[0])}_D{c[5]}_G{c[3] // c[4]}_"
+                         f"{'new' if c[6] else 'cached'}_s{c[7]}")
+def test_decode_parity(case):
+    lq, cache_lens, cache_len, hq, hkv, d, new, splits = case
+    cu_q, q, kc, vc, cs, kn, vn = _case(sum(cache_lens) + d, lq, cache_lens, cache_len, hq, hkv,
+                                        d, new)
+    kcd, vcd = kc.cuda(), vc.cuda()
+    scale = 1.0 / np.sqrt(d)
+    out, lse = va.varlen_attn_decode(q.cuda(), cu_q.cuda(), max(lq), kcd, vcd, cs.cuda(),
+                                     None if kn is None else kn.cuda(),
+                                     None if vn is None else vn.cuda(), softmax_scale=scale,
+                                     causal=True, num_splits=splits)
+    torch.cuda.synchronize()
+    exp_k = _expected_cache(kc, cs, cu_q, kn)
+    exp_v = _expected_cache(vc, cs, cu_q, vn)
+    assert torch.equal(kcd.cpu().view(torch.int16), exp_k.view(torch.int16))
+    assert torch.equal(vcd.cpu().view(torch.int16), exp_v.view(torch.int16))
+    lk = [cache_lens[i] + (lq[i] if new else 0) for i in range(len(lq))]
+    ref_o, ref_l = _oracle(q, cu_q, exp_k, exp_v, lk, hq, hkv, scale, True)
+    compare(out, lse, ref_o, ref_l)
+
+
+def test_decode_split_count_changes_only_rounding_and_is_deterministic():
+    lq, cache_lens = [1] * 6, [4000, 3000, 1, 2222, 4096, 100]
+    cu_q, q, kc, vc, cs, _, _ = _case(9, lq, cache_lens, 4096, 32, 8, 128, False)
+    args = (q.cuda(), cu_q.cuda(), 1, kc.cuda(), vc.cuda(), cs.cuda())
+    res = {}
+    for s in (1, 2, 5, 5):
+        o, l = va.varlen_attn_decode(*args, num_splits=s)
+        torch.cuda.synchronize()
+        if s in res:
+            assert torch.equal(o.view(torch.int16), res[s][0].view(torch.int16))
+            assert torch.equal(l.view(torch.int32), res[s][1].view(torch.int32))
+        res[s] = (o.clone(), l.clone())
+    for s in (2, 5):
+        assert (res[s][0].float() - res[1][0].float()).abs().max().item() < 2e-2
+        assert (res[s][1] - res[1][1]).abs().max().item() < 1e-4
+
+
+def test_decode_cache_overflow_reported():
+    cu_q = torch.tensor([0, 2], dtype=torch.int32, device="cuda")
+    q = torch.zeros(2, 4, 64, dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros(1, 8, 1, 64, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    kn = torch.ones(2, 1, 64, dtype=torch.bfloat16, device="cuda")
+    cs = torch.tensor([7], dtype=torch.int32, device="cuda")   # 7 + 2 new rows > 8
+    va.varlen_attn_decode(q, cu_q, 2, kc, vc, cs, kn, kn.clone())
+    assert va.get_device_error() == va.ERR_BAD_SEQLENS
+    assert torch.equal(kc[0, :7].cpu(), torch.zeros(7, 1, 64, dtype=torch.bfloat16))
