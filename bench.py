@@ -525,6 +525,68 @@ def run_layout(args, world, rank, local):
                          "peak_source": f"{src} hbm_gbs"}}), flush=True)
 
 
+def run_decode(args, world, rank, local):
+    """K/V-cache decode step: 64 sequences, one new query token each, cached
+    lengths U[1024, 8192] in a [64, 8192, 8, 128] bf16 cache (32/8 heads, the
+    long workload's head split). HBM-bound: reported as GB/s of the bytes a
+    step must move (cached K and V of every sequence once, q, out, LSE)
+    against the measured HBM peak."""
+    import torch
+    import packed_variable_length_attn_b200 as va
+    if rank != 0:
+        return
+    torch.cuda.set_device(local)
+    g = torch.Generator("cpu").manual_seed(20261299)
+    B, S, Hq, Hkv, D = 64, 8192, 32, 8, 128
+    lens = torch.randint(1024, 8192 + 1, (B,), generator=g).to(torch.int32)
+    if args.sequences and args.sequences < B:  # small case for profiling
+        B = args.sequences
+        lens = lens[:B]
+    dev = torch.device("cuda", local)
+    kc = torch.randn(B, S, Hkv, D, generator=g).to(torch.bfloat16).to(dev)
+    vc = torch.randn(B, S, Hkv, D, generator=g).to(torch.bfloat16).to(dev)
+    q = torch.randn(B, Hq, D, generator=g).to(torch.bfloat16).to(dev)
+    cu_q = torch.arange(B + 1, dtype=torch.int32, device=dev)
+    cs = lens.to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(Hq, B, dtype=torch.float32, device=dev)
+    nbytes = int(lens.sum()) * Hkv * D * 2 * 2 + 2 * q.numel() * 2 + lse.numel() * 4
+
+    def step():
+        va.varlen_attn_decode(q, cu_q, 1, kc, vc, cs, num_splits=args.decode_splits,
+                              out=out, lse=lse)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    # cache (8.6 GB) larger than L2: no flush needed between steps
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / args.steps
+    if va.get_device_error() != 0:
+        raise RuntimeError("device error in decode")
+    peaks, src = _peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    print(json.dumps({
+        "metric": "kv-cache decode step GB/s on 1 B200", "value": gbs, "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 cache and queries; cached lengths U[1024, 8192])",
+        "config": {"workload": "kv_cache_decode", "sequences": B, "q_len": 1, "cache_len": S,
+                   "cached_tokens": int(lens.sum()), "n_heads": Hq, "n_kv_heads": Hkv,
+                   "head_dim": D, "num_splits": args.decode_splits or "auto",
+                   "l2": "cache 8.6 GB > 126 MB L2; no flush"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]),
+                     "unit": "GB/s", "frac": gbs / float(peaks["hbm_gbs"]),
+                     "algorithmic_bytes_per_step": nbytes, "traffic": None,
+                     "peak_source": f"{src} hbm_gbs"}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -541,6 +603,10 @@ def main():
                     help="named workload (default: the long causal GQA workload)")
     ap.add_argument("--flush-l2", action="store_true",
                     help="256 MB scrub write between timed steps; each call timed alone")
+    ap.add_argument("--decode", action="store_true",
+                    help="time a K/V-cache decode step instead of the forward")
+    ap.add_argument("--decode-splits", type=int, default=0,
+                    help="--decode: key splits per (sequence, K/V head); 0 = automatic")
     ap.add_argument("--layout", action="store_true",
                     help="time the packed-layout helpers (unpad, pad) instead of the forward")
     ap.add_argument("--sequences", type=int, default=0,
@@ -552,6 +618,9 @@ def main():
         return
     if args.layout:
         run_layout(args, world, rank, local)
+        return
+    if args.decode:
+        run_decode(args, world, rank, local)
         return
     run_gpu(args, world, rank, local)
 

@@ -11,7 +11,10 @@ ROOT = os.path.dirname(HERE)
 SRC_DIR = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libvarlen_attn.so")
 SOURCES = ["varlen_attn.cu"]
-HEADERS = ["attn_sm100.cuh", "attn_f32.cuh", "sched.cuh", "common.cuh", "ptx.cuh"]
+# Every header the translation unit includes (a stale library is rebuilt when
+# any of them changes); checked against the csrc directory below.
+HEADERS = ["attn_sm100.cuh", "attn_f32.cuh", "sched.cuh", "common.cuh", "ptx.cuh", "layout.cuh",
+           "decode.cuh"]
 
 
 def nvcc_path() -> str:
@@ -22,7 +25,11 @@ def nvcc_path() -> str:
 
 
 def _inputs():
-    files = [os.path.join(SRC_DIR, f) for f in SOURCES + HEADERS]
+    # the listed files plus anything else in csrc, so a new header can never
+    # leave a stale library behind
+    names = set(SOURCES + HEADERS)
+    names |= {f for f in os.listdir(SRC_DIR) if f.endswith((".cu", ".cuh"))}
+    files = [os.path.join(SRC_DIR, f) for f in sorted(names)]
     files.append(os.path.join(ROOT, "include", "varlen_attn.h"))
     return files
 

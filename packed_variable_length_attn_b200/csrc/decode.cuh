@@ -23,9 +23,9 @@
 namespace va {
 
 constexpr int kDecThreads = 256;
-constexpr int kDecKeys = 64;     // keys per block of the ring
+constexpr int kDecKeys = 32;     // keys per block of the ring (one per lane in the softmax)
+constexpr int kDecStages = 2;    // ring depth: one block in flight while one is used
 constexpr int kDecMaxRows = 32;  // q_len x G rows per CTA
-constexpr int kDecMaxOut = kDecMaxRows * 128 / kDecThreads;  // O accumulators per thread
 
 struct DecodeParams {
   const __nv_bfloat16* q;       // [Tq, Hq, D]
@@ -43,6 +43,11 @@ struct DecodeParams {
   float* part_lse;              // [n_splits, Hq, Tq]
   int* error;
 };
+
+// bf16 -> fp32 is exact: the bf16 bits are the upper half of the fp32 bits.
+// Integer shifts / masks keep the conversions off the XU pipe.
+__device__ __forceinline__ float bf16_lo(uint32_t two) { return __uint_as_float(two << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t two) { return __uint_as_float(two & 0xffff0000u); }
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
@@ -82,26 +87,46 @@ __global__ void __launch_bounds__(kDecThreads) decode_append_kernel(DecodeParams
   }
 }
 
-template <int D>
+template <int D, int RT>
 struct DecSmem {
-  static constexpr int kKV = kDecKeys * D;                   // bf16 elements per block
-  static constexpr int kBytes = 2 * 2 * kKV * 2              // K and V, double-buffered
-                                + kDecMaxRows * D * 4        // Q (fp32)
-                                + kDecMaxRows * kDecKeys * 4 // scores / P
-                                + 3 * kDecMaxRows * 4;       // m, l, rescale factor
+  // K rows are padded by 64 bytes: with the interleaved dim slices of the
+  // score pass (thread c of a key reads dims 32m + 4c .. +3), the four keys a
+  // warp covers then fall on alternate bank halves and each 8-byte load
+  // instruction takes the minimum two wavefronts.
+  static constexpr int kKS = D + 32;        // K row stride (bf16 elements)
+  static constexpr int kKV = kDecKeys * kKS;  // bf16 elements per K (or V) block slot
+  // K and V ring (kDecStages blocks) | Q [RT][D] fp32 | P [kDecKeys][RT] fp32 | m, l, f [RT]
+  static constexpr int kKVBytes = kDecStages * 2 * kKV * 2;
+  static constexpr int kBytes = kKVBytes + RT * D * 4 + kDecKeys * RT * 4 + 3 * RT * 4;
+  static_assert(RT * D * 4 <= kKVBytes, "the final O reduction reuses the K/V buffers");
 };
 
-template <int D>
-__global__ void __launch_bounds__(kDecThreads) decode_kernel(DecodeParams p) {
+// One CTA: key split blockIdx.x of K/V head blockIdx.y of sequence blockIdx.z;
+// RT >= q_len * G query rows (rho = r * G + hl: query token r, head g*G + hl).
+// Per 64-key block:
+//   scores  8 threads per key, each a D/8 slice of the dot products of all
+//           rows with that key (the key is read once and used RT times),
+//           reduced over the 8 threads with shuffles;
+//   softmax one warp per row (online max / sum over the block);
+//   P V     each thread two output dims of every row, over its group of
+//           keys; the key groups' partial O are added once at the end.
+template <int D, int RT>
+__global__ void __launch_bounds__(kDecThreads, RT <= 8 ? 4 : 2) decode_kernel(DecodeParams p) {
   extern __shared__ __align__(16) uint8_t dsm[];
-  using S = DecSmem<D>;
-  __nv_bfloat16* kbuf = reinterpret_cast<__nv_bfloat16*>(dsm);            // [2][64][D]
-  __nv_bfloat16* vbuf = kbuf + 2 * S::kKV;                                 // [2][64][D]
-  float* qs = reinterpret_cast<float*>(vbuf + 2 * S::kKV);                 // [R][D]
-  float* ps = qs + kDecMaxRows * D;                                        // [R][64]
-  float* m_s = ps + kDecMaxRows * kDecKeys;
-  float* l_s = m_s + kDecMaxRows;
-  float* f_s = l_s + kDecMaxRows;
+  using S = DecSmem<D, RT>;
+  constexpr int kTPK = 8;                       // threads per key (scores)
+  constexpr int kDPT = D / kTPK;                // dims per thread (16 or 8)
+  constexpr int kKPP = kDecThreads / kTPK;      // keys per score pass (32)
+  constexpr int kNPair = D / 2;                 // output dim pairs (64 or 32)
+  constexpr int kNKG = kDecThreads / kNPair;    // key groups in P V (4 or 8)
+  constexpr int kKPG = kDecKeys / kNKG;         // keys per group (16 or 8)
+  __nv_bfloat16* kbuf = reinterpret_cast<__nv_bfloat16*>(dsm);            // [stages][64][D]
+  __nv_bfloat16* vbuf = kbuf + kDecStages * S::kKV;                        // [stages][64][D]
+  float* qs = reinterpret_cast<float*>(vbuf + kDecStages * S::kKV);        // [RT][D]
+  float* ps = qs + RT * D;                                                 // [64][RT]
+  float* m_s = ps + kDecKeys * RT;
+  float* l_s = m_s + RT;
+  float* f_s = l_s + RT;
 
   const int split = blockIdx.x, g = blockIdx.y, i = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -110,7 +135,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(DecodeParams p) {
   const int R = Lq * G;
   if (Lq <= 0) return;
   const int Lk = p.cache_seqlens[i] + (p.k_new ? Lq : 0);
-  if (R > kDecMaxRows || Lk > p.cache_len || Lk < 0) {
+  if (R > RT || Lk > p.cache_len || Lk < 0) {
     if (tid == 0) atomicCAS(p.error, 0, kErrBadSeqlens);
     return;
   }
@@ -119,19 +144,23 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(DecodeParams p) {
   const int per = (nblk_all + p.n_splits - 1) / p.n_splits;
   const int b0 = split * per, b1 = min(nblk_all, b0 + per);
 
-  // rows: rho = r * G + hl (query token r, query head g*G + hl)
-  for (int e = tid; e < R * D; e += kDecThreads) {
+  for (int e = tid; e < RT * D; e += kDecThreads) {
     const int rho = e / D, d = e - rho * D;
-    const int r = rho / G, hl = rho - r * G;
-    qs[e] = __bfloat162float(p.q[((long long)(q0 + r) * p.n_heads + g * G + hl) * D + d]);
+    float v = 0.f;
+    if (rho < R) {
+      const int r = rho / G, hl = rho - r * G;
+      v = __bfloat162float(p.q[((long long)(q0 + r) * p.n_heads + g * G + hl) * D + d]);
+    }
+    qs[e] = v;
   }
-  for (int rho = tid; rho < kDecMaxRows; rho += kDecThreads) {
+  for (int rho = tid; rho < RT; rho += kDecThreads) {
     m_s[rho] = -INFINITY;
     l_s[rho] = 0.f;
   }
-  float acc[kDecMaxOut];
+  const int dp = tid % kNPair, kg = tid / kNPair;  // P V: dims 2dp, 2dp+1; key group kg
+  float acc[RT][2];
 #pragma unroll
-  for (int j = 0; j < kDecMaxOut; ++j) acc[j] = 0.f;
+  for (int rho = 0; rho < RT; ++rho) acc[rho][0] = acc[rho][1] = 0.f;
 
   const long long row_stride = (long long)p.n_kv_heads * D;  // elements between cache rows
   const __nv_bfloat16* kbase = p.k_cache + (long long)i * p.cache_len * row_stride + (long long)g * D;
@@ -141,8 +170,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(DecodeParams p) {
     const int k0 = blk * kDecKeys;
     for (int e = tid; e < kDecKeys * kUnitsPerRow; e += kDecThreads) {
       const int kr = e / kUnitsPerRow, u = e - kr * kUnitsPerRow;
-      __nv_bfloat16* kd = kbuf + buf * S::kKV + kr * D + u * 8;
-      __nv_bfloat16* vd = vbuf + buf * S::kKV + kr * D + u * 8;
+      __nv_bfloat16* kd = kbuf + buf * S::kKV + kr * S::kKS + u * 8;
+      __nv_bfloat16* vd = vbuf + buf * S::kKV + kr * S::kKS + u * 8;
       if (k0 + kr < Lk) {
         cp_async16(kd, kbase + (long long)(k0 + kr) * row_stride + u * 8);
         cp_async16(vd, vbase + (long long)(k0 + kr) * row_stride + u * 8);
@@ -152,57 +181,83 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(DecodeParams p) {
       }
     }
   };
-  if (b0 < b1) load_block(b0, 0);
-  cp_async_commit();
+#pragma unroll
+  for (int st = 0; st < kDecStages - 1; ++st) {
+    if (b0 + st < b1) load_block(b0 + st, st);
+    cp_async_commit();
+  }
   __syncthreads();  // Q, m, l visible
 
   for (int blk = b0; blk < b1; ++blk) {
-    const int buf = (blk - b0) & 1;
-    if (blk + 1 < b1) load_block(blk + 1, buf ^ 1);
+    const int buf = (blk - b0) % kDecStages;
+    const int ahead = blk + kDecStages - 1;
+    if (ahead < b1) load_block(ahead, (ahead - b0) % kDecStages);
     cp_async_commit();
-    cp_async_wait<1>();
+    cp_async_wait<kDecStages - 1>();  // block blk has landed
     __syncthreads();
     const __nv_bfloat16* kb = kbuf + buf * S::kKV;
     const __nv_bfloat16* vb = vbuf + buf * S::kKV;
     const int k0 = blk * kDecKeys;
-    // scores (log2 domain): thread -> (row, key); the d loop starts at a
-    // key-dependent offset so that the 32 keys of a warp hit 32 banks.
-    for (int e = tid; e < R * kDecKeys; e += kDecThreads) {
-      const int rho = e / kDecKeys, kr = e - rho * kDecKeys;
-      const int r = rho / G;
-      const int c = k0 + kr;
-      float s = -INFINITY;
-      const bool visible = c < Lk && (!p.causal || c <= r + Lk - Lq);
-      if (visible) {
-        const __nv_bfloat162* krow = reinterpret_cast<const __nv_bfloat162*>(kb + kr * D);
-        const float2* qrow = reinterpret_cast<const float2*>(qs + rho * D);
-        float a0 = 0.f, a1 = 0.f;
-#pragma unroll 8
-        for (int m = 0; m < D / 2; ++m) {
-          const int mm = (m + kr) & (D / 2 - 1);
-          const float2 kv = __bfloat1622float2(krow[mm]);
-          const float2 qv = qrow[mm];
-          a0 = fmaf(qv.x, kv.x, a0);
-          a1 = fmaf(qv.y, kv.y, a1);
-        }
-        s = (a0 + a1) * p.scale_log2;
+    // scores (log2 domain); thread c of a key holds dims 32m + 4c .. 32m + 4c + 3
+#pragma unroll
+    for (int pass = 0; pass < kDecKeys / kKPP; ++pass) {
+      const int kr = pass * kKPP + tid / kTPK, c = tid % kTPK;
+      float kf[kDPT];
+#pragma unroll
+      for (int m = 0; m < D / 32; ++m) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(kb + kr * S::kKS + 32 * m + 4 * c);
+        kf[4 * m] = bf16_lo(raw.x);
+        kf[4 * m + 1] = bf16_hi(raw.x);
+        kf[4 * m + 2] = bf16_lo(raw.y);
+        kf[4 * m + 3] = bf16_hi(raw.y);
       }
-      ps[rho * kDecKeys + kr] = s;
+      const int key = k0 + kr;
+#pragma unroll 1
+      for (int r0 = 0; r0 < RT; r0 += 4) {  // four rows at a time (bounded registers)
+        float part[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float* qrow = qs + (r0 + j) * D + 4 * c;
+          float a = 0.f, b = 0.f;
+#pragma unroll
+          for (int m = 0; m < D / 32; ++m) {
+            const float4 qv = *reinterpret_cast<const float4*>(qrow + 32 * m);
+            a = fmaf(qv.x, kf[4 * m], a);
+            b = fmaf(qv.y, kf[4 * m + 1], b);
+            a = fmaf(qv.z, kf[4 * m + 2], a);
+            b = fmaf(qv.w, kf[4 * m + 3], b);
+          }
+          part[j] = a + b;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+#pragma unroll
+          for (int o = 1; o < kTPK; o <<= 1) part[j] += __shfl_xor_sync(0xffffffffu, part[j], o);
+        }
+        if (c == 0) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int rho = r0 + j, r = rho / G;
+            const bool vis = rho < R && key < Lk && (!p.causal || key <= r + Lk - Lq);
+            ps[kr * RT + rho] = vis ? part[j] * p.scale_log2 : -INFINITY;
+          }
+        }
+      }
     }
     __syncthreads();
-    // online softmax: one warp per row, two keys per lane
+    // online softmax: one warp per row, one key per lane
+    static_assert(kDecKeys == 32, "one key per lane");
     for (int rho = warp; rho < R; rho += kDecThreads / 32) {
-      const float s0 = ps[rho * kDecKeys + lane], s1 = ps[rho * kDecKeys + lane + 32];
-      float mx = fmaxf(s0, s1);
+      const float s0 = ps[lane * RT + rho];
+      float mx = s0;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       const float m_old = m_s[rho];
       const float m_new = fmaxf(m_old, mx);
       const float mb = m_new == -INFINITY ? 0.f : m_new;
-      const float e0 = exp2f(s0 - mb), e1 = exp2f(s1 - mb);
-      ps[rho * kDecKeys + lane] = e0;
-      ps[rho * kDecKeys + lane + 32] = e1;
-      float sum = e0 + e1;
+      const float e0 = exp2f(s0 - mb);
+      ps[lane * RT + rho] = e0;
+      float sum = e0;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
       if (lane == 0) {
@@ -212,39 +267,68 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(DecodeParams p) {
         m_s[rho] = m_new;
       }
     }
+    for (int rho = R + tid; rho < RT; rho += kDecThreads) {  // rows past R: no contribution
+      f_s[rho] = 0.f;
+      for (int kk = 0; kk < kDecKeys; ++kk) ps[kk * RT + rho] = 0.f;
+    }
     __syncthreads();
-    // O = O * fac + P V: thread -> outputs (row, d) = e, e + 256, ...
+    // O = O * fac + P V over this thread's key group
 #pragma unroll
-    for (int j = 0; j < kDecMaxOut; ++j) {
-      const int e = tid + j * kDecThreads;
-      if (e < R * D) {
-        const int rho = e / D, d = e - rho * D;
-        float a = acc[j] * f_s[rho];
-        const float* prow = ps + rho * kDecKeys;
-#pragma unroll 8
-        for (int kr = 0; kr < kDecKeys; ++kr) a = fmaf(prow[kr], __bfloat162float(vb[kr * D + d]), a);
-        acc[j] = a;
+    for (int rho = 0; rho < RT; ++rho) {
+      const float f = f_s[rho];
+      acc[rho][0] *= f;
+      acc[rho][1] *= f;
+    }
+#pragma unroll 4
+    for (int kk = 0; kk < kKPG; ++kk) {
+      const int key = kg * kKPG + kk;
+      const uint32_t vraw = *reinterpret_cast<const uint32_t*>(vb + key * S::kKS + 2 * dp);
+      const float2 v = make_float2(bf16_lo(vraw), bf16_hi(vraw));
+      const float4* prow = reinterpret_cast<const float4*>(ps + key * RT);
+#pragma unroll
+      for (int r4 = 0; r4 < RT / 4; ++r4) {
+        const float4 pv = prow[r4];
+        acc[4 * r4][0] = fmaf(pv.x, v.x, acc[4 * r4][0]);
+        acc[4 * r4][1] = fmaf(pv.x, v.y, acc[4 * r4][1]);
+        acc[4 * r4 + 1][0] = fmaf(pv.y, v.x, acc[4 * r4 + 1][0]);
+        acc[4 * r4 + 1][1] = fmaf(pv.y, v.y, acc[4 * r4 + 1][1]);
+        acc[4 * r4 + 2][0] = fmaf(pv.z, v.x, acc[4 * r4 + 2][0]);
+        acc[4 * r4 + 2][1] = fmaf(pv.z, v.y, acc[4 * r4 + 2][1]);
+        acc[4 * r4 + 3][0] = fmaf(pv.w, v.x, acc[4 * r4 + 3][0]);
+        acc[4 * r4 + 3][1] = fmaf(pv.w, v.y, acc[4 * r4 + 3][1]);
       }
     }
-    __syncthreads();  // the buffer is reloaded two blocks later; ps, f_s reused
+    __syncthreads();  // this stage is reloaded by the next iteration; ps, f_s reused
   }
   cp_async_wait<0>();
+  __syncthreads();
+
+  // add the key groups' partial O in a fixed order (deterministic), in the
+  // now free K/V buffers: O [RT][D] fp32
+  float* osum = reinterpret_cast<float*>(dsm);
+  for (int grp = 0; grp < kNKG; ++grp) {
+    if (kg == grp) {
+#pragma unroll
+      for (int rho = 0; rho < RT; ++rho) {
+        float2* dst = reinterpret_cast<float2*>(osum + rho * D + 2 * dp);
+        const float2 prev = grp == 0 ? make_float2(0.f, 0.f) : *dst;
+        *dst = make_float2(prev.x + acc[rho][0], prev.y + acc[rho][1]);
+      }
+    }
+    __syncthreads();
+  }
 
   // epilogue: normalise; one split writes the result, several write partials
-#pragma unroll
-  for (int j = 0; j < kDecMaxOut; ++j) {
-    const int e = tid + j * kDecThreads;
-    if (e < R * D) {
-      const int rho = e / D, d = e - rho * D;
-      const int r = rho / G, h = g * G + (rho - r * G);
-      const float l = l_s[rho];
-      const float o = l > 0.f ? acc[j] / l : 0.f;
-      const long long oi = ((long long)(q0 + r) * p.n_heads + h) * D + d;
-      if (p.n_splits == 1)
-        p.out[oi] = __float2bfloat16_rn(o);
-      else
-        p.part_o[(long long)split * p.total_q * p.n_heads * D + oi] = o;
-    }
+  for (int e = tid; e < R * D; e += kDecThreads) {
+    const int rho = e / D, d = e - rho * D;
+    const int r = rho / G, h = g * G + (rho - r * G);
+    const float l = l_s[rho];
+    const float o = l > 0.f ? osum[e] / l : 0.f;
+    const long long oi = ((long long)(q0 + r) * p.n_heads + h) * D + d;
+    if (p.n_splits == 1)
+      p.out[oi] = __float2bfloat16_rn(o);
+    else
+      p.part_o[(long long)split * p.total_q * p.n_heads * D + oi] = o;
   }
   for (int rho = tid; rho < R; rho += kDecThreads) {
     const int r = rho / G, h = g * G + (rho - r * G);

@@ -381,6 +381,14 @@ int rows_args_ok(const void* src, int64_t src_rows, int64_t row_bytes, const int
   return VARLEN_ATTN_OK;
 }
 
+template <int D, int RT>
+int launch_decode(dim3 grid, const DecodeParams& dp, cudaStream_t st) {
+  auto kern = decode_kernel<D, RT>;
+  if (int rc = set_smem(kern, DecSmem<D, RT>::kBytes)) return rc;
+  kern<<<grid, kDecThreads, DecSmem<D, RT>::kBytes, st>>>(dp);
+  return check_launch("launch decode_kernel");
+}
+
 }  // namespace
 
 extern "C" {
@@ -719,13 +727,15 @@ int varlen_attn_decode(const void* q, const int32_t* cu_seqlens_q, int batch, in
   if (int rc = device_info(&di)) return rc;
   if (total_q == 0 || max_seqlen_q == 0) return VARLEN_ATTN_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // splits: enough CTAs for two per SM, each split at least 256 keys
+  // splits: about 16 CTAs per SM over the whole grid (several waves keep the
+  // SMs busy despite unequal cache lengths), each split at least 256 keys
   int splits = num_splits;
   const int max_blocks = (cache_len + kDecKeys - 1) / kDecKeys;
   if (splits == 0) {
     const int64_t ctas = (int64_t)batch * n_kv_heads;
-    const int64_t want = (2 * (int64_t)di->sm_count + ctas - 1) / ctas;
-    splits = (int)std::max<int64_t>(1, std::min<int64_t>(want, std::max(1, max_blocks / 4)));
+    const int64_t want = (16 * (int64_t)di->sm_count + ctas - 1) / ctas;
+    const int min_blocks = (256 + kDecKeys - 1) / kDecKeys;
+    splits = (int)std::max<int64_t>(1, std::min<int64_t>(want, std::max(1, max_blocks / min_blocks)));
   }
   splits = std::min(splits, std::max(1, max_blocks));
   DecodeParams dp;
@@ -761,27 +771,35 @@ int varlen_attn_decode(const void* q, const int32_t* cu_seqlens_q, int batch, in
   const dim3 grid(splits, n_kv_heads, batch);
   const int rows = (int)std::min<int64_t>((int64_t)total_q * n_heads / (kDecThreads / 32) + 1,
                                           (int64_t)di->sm_count * 16);
-  if (head_dim == 64) {
-    if (k_new) {
-      decode_append_kernel<64><<<layout_grid(di, (int64_t)total_q * n_kv_heads * 8), kDecThreads,
-                                 0, st>>>(dp);
-      if (int rc = check_launch("launch decode_append_kernel")) return rc;
-    }
-    if (int rc = set_smem(decode_kernel<64>, DecSmem<64>::kBytes)) return rc;
-    decode_kernel<64><<<grid, kDecThreads, DecSmem<64>::kBytes, st>>>(dp);
-    if (int rc = check_launch("launch decode_kernel")) return rc;
-    if (splits > 1) decode_combine_kernel<64><<<rows, kDecThreads, 0, st>>>(dp);
-  } else {
-    if (k_new) {
-      decode_append_kernel<128><<<layout_grid(di, (int64_t)total_q * n_kv_heads * 16),
-                                  kDecThreads, 0, st>>>(dp);
-      if (int rc = check_launch("launch decode_append_kernel")) return rc;
-    }
-    if (int rc = set_smem(decode_kernel<128>, DecSmem<128>::kBytes)) return rc;
-    decode_kernel<128><<<grid, kDecThreads, DecSmem<128>::kBytes, st>>>(dp);
-    if (int rc = check_launch("launch decode_kernel")) return rc;
-    if (splits > 1) decode_combine_kernel<128><<<rows, kDecThreads, 0, st>>>(dp);
+  if (k_new) {
+    const int units = n_kv_heads * head_dim / 8;
+    if (head_dim == 64)
+      decode_append_kernel<64><<<layout_grid(di, (int64_t)total_q * units), kDecThreads, 0, st>>>(dp);
+    else
+      decode_append_kernel<128><<<layout_grid(di, (int64_t)total_q * units), kDecThreads, 0, st>>>(dp);
+    if (int rc = check_launch("launch decode_append_kernel")) return rc;
   }
+  const int rows_needed = max_seqlen_q * G;
+  const int RT = rows_needed <= 4 ? 4 : rows_needed <= 8 ? 8 : rows_needed <= 16 ? 16 : 32;
+  int rc = VARLEN_ATTN_OK;
+  if (head_dim == 64) {
+    switch (RT) {
+      case 4: rc = launch_decode<64, 4>(grid, dp, st); break;
+      case 8: rc = launch_decode<64, 8>(grid, dp, st); break;
+      case 16: rc = launch_decode<64, 16>(grid, dp, st); break;
+      default: rc = launch_decode<64, 32>(grid, dp, st); break;
+    }
+    if (!rc && splits > 1) decode_combine_kernel<64><<<rows, kDecThreads, 0, st>>>(dp);
+  } else {
+    switch (RT) {
+      case 4: rc = launch_decode<128, 4>(grid, dp, st); break;
+      case 8: rc = launch_decode<128, 8>(grid, dp, st); break;
+      case 16: rc = launch_decode<128, 16>(grid, dp, st); break;
+      default: rc = launch_decode<128, 32>(grid, dp, st); break;
+    }
+    if (!rc && splits > 1) decode_combine_kernel<128><<<rows, kDecThreads, 0, st>>>(dp);
+  }
+  if (rc) return rc;
   return check_launch("launch decode_combine_kernel");
 }
 
