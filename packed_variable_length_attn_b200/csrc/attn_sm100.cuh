@@ -74,7 +74,11 @@ struct KCfg {
   static constexpr int kBiasOff = kKVOff + kStages * kKVTile;  // float [2 slot][2 buf][BN]
   static constexpr int kEpiOff = kBiasOff + 2 * 2 * BN * 4;     // O staging: 2 KB per softmax warp
   static constexpr int kEpiWarpBytes = 32 * 32 * 2;             // 32 rows x 32 bf16 columns
-  static constexpr int kItemOff = kEpiOff + 8 * kEpiWarpBytes;
+  // Pair-grid staging ring per softmax warp: the O staging block plus
+  // kPairBufs - 1 more blocks of the same size (head_dim 64 has the room).
+  static constexpr int kPairBufs = D == 64 ? 3 : 1;
+  static constexpr int kPairOff = kEpiOff + 8 * kEpiWarpBytes;
+  static constexpr int kItemOff = kPairOff + 8 * (kPairBufs - 1) * kEpiWarpBytes;
   static constexpr int kBarOff = kItemOff + ((2 * (int)sizeof(Item) + 15) / 16) * 16;
   // barriers: q_full[2] q_empty[2] s_full[2] p_full[2][2 halves] o_full[2]
   //           o_empty[2] item_full[2] item_empty[2] bias_full[2][2] drain
@@ -157,6 +161,11 @@ struct Smem {
     return reinterpret_cast<float*>(base + KCfg<D>::kBiasOff) + (s * 2 + b) * BN;
   }
   __device__ uint8_t* epi(int warp) const { return base + KCfg<D>::kEpiOff + warp * KCfg<D>::kEpiWarpBytes; }
+  // pair-grid staging block b of a softmax warp (block 0 is its O staging)
+  __device__ uint8_t* pair_buf(int warp, int b) const {
+    return b == 0 ? epi(warp)
+                  : base + KCfg<D>::kPairOff + (warp * (KCfg<D>::kPairBufs - 1) + b - 1) * KCfg<D>::kEpiWarpBytes;
+  }
   __device__ Item* items() const { return reinterpret_cast<Item*>(base + KCfg<D>::kItemOff); }
   __device__ uint64_t* bars() const { return reinterpret_cast<uint64_t*>(base + KCfg<D>::kBarOff); }
   __device__ uint64_t* q_full(int s) const { return bars() + 0 + s; }
@@ -447,9 +456,11 @@ __device__ __forceinline__ void rescale_o(uint32_t t_o, float fac) {
 }
 
 // ------------------------------------------------------------------ softmax
+
 template <int D, bool kBiasKey, bool kBiasPair>
 __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams& p,
                              const Ctl& ctl) {
+  using C = KCfg<D>;
   const int warp = threadIdx.x >> 5;
   const int wg = warp >> 2;                    // slot
   const int r = threadIdx.x & 127;             // tile row = TMEM lane
@@ -484,10 +495,6 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
     const int q_loc = q_loc0 + r;
     const bool row_ok = r < rows;
     const int limit = p.causal ? min(Lk, q_loc + (Lk - Lq) + 1) : Lk;
-    const float* brow = nullptr;
-    if (kBiasPair && row_ok)
-      brow = p.bias_pair + (long long)seq * p.sb + (long long)(head / p.bias_head_div) * p.sh +
-             (long long)q_loc * p.sr;
     float m_used = -INFINITY, l = 0.f;
 
     for (int j = 0; j < n; ++j) {
@@ -499,9 +506,42 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
       if constexpr (kBiasKey) {
         bk = sm.bias(wg, b);
         const int key = kb + r;
-        bk[r] = key < Lk ? p.bias_key[(long long)(kv_row0 + key) * p.n_heads + head] * kLog2e
-                         : 0.f;
+        bk[r] = key < Lk ? p.bias_key[(long long)(kv_row0 + key) * p.n_heads + head] : 0.f;
         ptx::mbar_arrive(sm.bias_full(wg, b));
+      }
+      // Pair grid, 16-byte rows: the warp's 32 rows x 128 keys arrive in
+      // chunks of 16 keys (2 KB) through a ring of kPairBufs staging blocks,
+      // copied straight to shared memory (cp.async, coalesced: 4 lanes per
+      // 64-byte row piece, 8 rows per instruction). The first chunks are in
+      // flight while the scores are computed.
+      const int lane = threadIdx.x & 31;
+      const float* prow = nullptr;  // lane's row piece at key kb + 4 * (lane % 4)
+      auto pair_dst = [&](int b, int x, int cu) {
+        return ptx::smem_u32(sm.pair_buf(warp, b)) + (uint32_t)(4 * x + (cu ^ ((x >> 1) & 3))) * 16u;
+      };
+      auto pair_issue = [&](int ch) {
+        if (ch < BN / 16) {
+          const int key0 = kb + ch * 16 + 4 * (lane & 3);
+          const int kleft = Lk - key0;
+          const uint32_t nb = kleft >= 4 ? 16u : kleft > 0 ? 4u * (uint32_t)kleft : 0u;
+#pragma unroll
+          for (int k8 = 0; k8 < 4; ++k8) {
+            const int x = 8 * k8 + (lane >> 2);
+            const bool in = (warp & 3) * 32 + x < rows && nb > 0;
+            const float* src = in ? prow + (long long)(8 * k8) * p.sr + ch * 16 : p.bias_pair;
+            ptx::cp_async16_zfill(pair_dst(ch % C::kPairBufs, x, lane & 3), src, in ? nb : 0u);
+          }
+        }
+        ptx::cp_async_commit_group();
+      };
+      if constexpr (kBiasPair) {
+        if (p.pair_vec) {
+          prow = p.bias_pair + (long long)seq * p.sb + (long long)(head / p.bias_head_div) * p.sh +
+                 (long long)(q_loc0 + (warp & 3) * 32 + (lane >> 2)) * p.sr + kb + 4 * (lane & 3);
+          __syncwarp();  // earlier reads of the staging blocks are done
+#pragma unroll
+          for (int ch = 0; ch < C::kPairBufs; ++ch) pair_issue(ch);
+        }
       }
       ok = __all_sync(FULL, wait_bar(sm.s_full(wg), ph, ctl));
       if (!ok) break;
@@ -518,36 +558,70 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
       for (int c = 0; c < BN / 32; ++c)
         ptx::tmem_ld32(t_s + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c * 32]));
       ptx::tmem_wait_ld();
-      const bool prescaled = kBiasKey || kBiasPair || !(p.scale_log2 > 0.f);
+      // With a bias the row holds natural-unit scores s * scale + bias (one
+      // packed FMA per pair of keys) and log2(e) goes into the exponent's
+      // FMA; without one, the raw scores stay and scale * log2(e) goes there
+      // (the scale commutes with the row max when it is positive).
+      constexpr bool kBiased = kBiasKey || kBiasPair;
+      const bool prescaled = !kBiased && !(p.scale_log2 > 0.f);
+      const uint64_t scale2 = ptx::f2(p.scale, p.scale);
       if (prescaled) {
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          float x;
-          if constexpr (kBiasKey)
-            x = fmaf(__uint_as_float(u[c]), p.scale_log2, bk[c]);
-          else
-            x = __uint_as_float(u[c]) * p.scale_log2;
-          u[c] = __float_as_uint(x);
+        for (int c = 0; c < BN; ++c) u[c] = __float_as_uint(__uint_as_float(u[c]) * p.scale_log2);
+      }
+      if constexpr (kBiasKey) {
+#pragma unroll
+        for (int c = 0; c < BN; c += 2) {
+          const float2 b2 = *reinterpret_cast<const float2*>(bk + c);
+          const uint64_t x2 = ptx::ffma2(ptx::f2(__uint_as_float(u[c]), __uint_as_float(u[c + 1])),
+                                         scale2, ptx::f2(b2.x, b2.y));
+          float lo, hi;
+          ptx::f2_split(x2, lo, hi);
+          u[c] = __float_as_uint(lo);
+          u[c + 1] = __float_as_uint(hi);
         }
       }
+      // Adds a pair of grid entries to a pair of scores: onto s * scale + key
+      // bias when there is a per-key bias, else onto the raw scores with the
+      // scale applied in the same packed FMA.
+      auto pair_add2 = [&](uint32_t& u0, uint32_t& u1, uint32_t b0, uint32_t b1, uint64_t sc2) {
+        const uint64_t s2 = ptx::f2(__uint_as_float(u0), __uint_as_float(u1));
+        const uint64_t g2 = ptx::f2(__uint_as_float(b0), __uint_as_float(b1));
+        const uint64_t x2 = kBiasKey ? ptx::fadd2(s2, g2) : ptx::ffma2(s2, sc2, g2);
+        float lo, hi;
+        ptx::f2_split(x2, lo, hi);
+        u0 = __float_as_uint(lo);
+        u1 = __float_as_uint(hi);
+      };
       if constexpr (kBiasPair) {
-        if (brow != nullptr) {
+        if (p.pair_vec) {
+#pragma unroll
+          for (int ch = 0; ch < BN / 16; ++ch) {
+            ptx::cp_async_wait_group<C::kPairBufs - 1>();  // chunk ch has landed
+            __syncwarp();
+#pragma unroll
+            for (int cu = 0; cu < 4; ++cu) {
+              const uint4 b = ptx::ld_shared_v4(pair_dst(ch % C::kPairBufs, lane, cu));
+              const int c = ch * 16 + 4 * cu;
+              pair_add2(u[c], u[c + 1], b.x, b.y, scale2);
+              pair_add2(u[c + 2], u[c + 3], b.z, b.w, scale2);
+            }
+            __syncwarp();  // block (ch % kPairBufs) is free again
+            pair_issue(ch + C::kPairBufs);
+          }
+        } else if (row_ok) {
+          const float* brow = p.bias_pair + (long long)seq * p.sb +
+                              (long long)(head / p.bias_head_div) * p.sh + (long long)q_loc * p.sr;
 #pragma unroll
           for (int c = 0; c < BN; c += 4) {
             const int key = kb + c;
-            if (p.pair_vec && key + 3 < Lk) {
-              const float4 b4 = __ldg(reinterpret_cast<const float4*>(brow + key));
-              u[c] = __float_as_uint(fmaf(b4.x, kLog2e, __uint_as_float(u[c])));
-              u[c + 1] = __float_as_uint(fmaf(b4.y, kLog2e, __uint_as_float(u[c + 1])));
-              u[c + 2] = __float_as_uint(fmaf(b4.z, kLog2e, __uint_as_float(u[c + 2])));
-              u[c + 3] = __float_as_uint(fmaf(b4.w, kLog2e, __uint_as_float(u[c + 3])));
-            } else {
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                if (key + e < Lk)
-                  u[c + e] = __float_as_uint(fmaf(__ldg(brow + (long long)(key + e) * p.sc),
-                                                  kLog2e, __uint_as_float(u[c + e])));
-            }
+            for (int e = 0; e < 4; ++e)
+              if (key + e < Lk) {
+                const float b = __ldg(brow + (long long)(key + e) * p.sc);
+                const float x = __uint_as_float(u[c + e]);
+                u[c + e] = __float_as_uint(kBiasKey ? x + b : fmaf(x, p.scale, b));
+              }
           }
         }
       }
@@ -568,7 +642,7 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
       mx[14] = mx[42];
 #pragma unroll
       for (int i = 0; i < 5; ++i) mx[i] = ptx::fmax3(mx[3 * i], mx[3 * i + 1], mx[3 * i + 2]);
-      const float sfac = prescaled ? 1.f : p.scale_log2;
+      const float sfac = kBiased ? kLog2e : prescaled ? 1.f : p.scale_log2;
       const float m_tile = ptx::fmax3(ptx::fmax3(mx[0], mx[1], mx[2]), mx[3], mx[4]) * sfac;
       const float m_new = fmaxf(m_used, m_tile);
       const bool need = m_new > m_used + kRescaleThreshold;
@@ -678,6 +752,7 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
       p.lse[(long long)head * p.total_q + q_row0 + r] = lse;
     }
   }
+  if constexpr (kBiasPair) ptx::cp_async_wait_group<0>();  // copies left by an abort
 }
 
 // ------------------------------------------------------------------ kernel

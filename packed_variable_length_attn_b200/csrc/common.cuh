@@ -47,6 +47,7 @@ struct AttnParams {
   int pairing, n_hp, n_hg;
   int causal;
   float scale_log2;                // softmax_scale * log2(e)
+  float scale;                     // softmax_scale
   const float* bias_key;           // [Tk, Hq] or null
   const float* bias_pair;          // strided grid or null
   long long sb, sh, sr, sc;

@@ -325,6 +325,7 @@ int fwd_bf16(const void* q, const void* k, const void* v, const int32_t* cu_seql
   prm.n_hg = n_hg;
   prm.causal = a.causal;
   prm.scale_log2 = softmax_scale * 1.4426950408889634f;
+  prm.scale = softmax_scale;
   prm.bias_key = bias_per_key;
   prm.bias_pair = bias_pair;
   prm.sb = bias_stride_b;
@@ -576,6 +577,7 @@ int varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   prm.n_hg = n_hg;
   prm.causal = a.causal;
   prm.scale_log2 = softmax_scale * 1.4426950408889634f;
+  prm.scale = softmax_scale;
   prm.bias_key = bias_per_key;
   prm.bias_pair = bias_pair;
   prm.sb = bias_stride_b;
