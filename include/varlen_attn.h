@@ -203,6 +203,51 @@ int varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                             void* out, float* lse, void* stream);
 
 /*
+ * Backward pass of varlen_attn_fwd (bf16). The gradients of a loss through
+ * O = varlen_attn_fwd(...): the packed path's gradients that the TorchEasyRec
+ * PR 663 page (GenRec, "Test plan") checks and the ASpec PR 25 page
+ * ("Verification") bounds at 1% relative L2 for Q/K/V, including the bias
+ * gradients that the GiGL PR 858 page ("Approach") lists as missing for a
+ * per-sequence bias. With P the forward's probabilities and
+ * delta = rowsum(dO * O):
+ *
+ *   dV = P^T dO,  dS = P * (dO V^T - delta),  dQ = scale dS K,  dK = scale dS^T Q,
+ *   dbias_per_key[cu_k[i] + c, h] = sum_r dS[r, c],  dbias_pair[i, h, r, c] = dS[r, c].
+ *
+ * Inputs: everything varlen_attn_fwd took (same meaning, same flags), plus
+ *   out  [total_q, n_heads, head_dim] bf16: the forward's output;
+ *   lse  [n_heads, total_q] fp32: the forward's LSE (required);
+ *   dout [total_q, n_heads, head_dim] bf16: the gradient of the loss w.r.t. out.
+ * Outputs (caller-owned, written, not accumulated):
+ *   dq [total_q, n_heads, head_dim], dk and dv [total_k, n_kv_heads, head_dim]
+ *   bf16 (dk, dv summed over the n_heads / n_kv_heads query heads of a group);
+ *   dbias_per_key [total_k, n_heads] fp32 or NULL (not computed);
+ *   dbias_pair fp32 or NULL: entry (i, h, r, c) at i*dbias_stride_b +
+ *   h*dbias_stride_h + r*dbias_stride_q + c for every query head h and every
+ *   in-sequence (r, c); other entries are left as they are. A broadcast or
+ *   per-K/V-head grid's gradient is the sum of these over the heads that read it.
+ * Rows without a visible key get zero gradients. Deterministic (no atomics):
+ * one launch validates cu_seqlens (a bad table raises VARLEN_ATTN_ERR_BAD_SEQLENS
+ * on the device and writes no gradient), one computes delta into the library
+ * workspace, one computes dK and dV per (sequence, K/V head, 128-key block),
+ * one dQ per (sequence, query head, 128-row block). Errors as for
+ * varlen_attn_fwd; batch or n_heads above 65535: VARLEN_ATTN_ERR_TOO_LARGE.
+ */
+int varlen_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                    const float* lse, const void* dout,
+                    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                    int batch, int total_q, int total_k,
+                    int max_seqlen_q, int max_seqlen_k,
+                    int n_heads, int n_kv_heads, int head_dim,
+                    float softmax_scale, int causal,
+                    const float* bias_per_key,
+                    const float* bias_pair, int64_t bias_stride_b, int64_t bias_stride_h,
+                    int64_t bias_stride_q, int64_t bias_stride_k, unsigned flags,
+                    void* dq, void* dk, void* dv, float* dbias_per_key,
+                    float* dbias_pair, int64_t dbias_stride_b, int64_t dbias_stride_h,
+                    int64_t dbias_stride_q, void* stream);
+
+/*
  * Decode attention over a per-sequence K/V cache (flash_attn_with_kvcache in
  * "fix(flex): avoid decoding kernel selection for short GQA" and the noether
  * attention module page; q_len = 1 decode steps, FDMA integration page,

@@ -24,7 +24,7 @@ from typing import Optional, Sequence, Tuple
 __all__ = ["varlen_attn_fwd", "varlen_attn_fwd_noalloc", "library_path", "load_library", "VarlenAttnError",
            "get_device_error", "set_profile_events", "launches_per_call", "exported_symbols",
            "mask_to_seqlens", "gather_rows", "scatter_rows", "unpad", "pad", "fold_pair_bias_row",
-           "varlen_attn_decode", "BIAS_PAIR_KV_HEADS"]
+           "varlen_attn_decode", "varlen_attn_bwd", "BIAS_PAIR_KV_HEADS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libvarlen_attn.so")
@@ -53,7 +53,7 @@ def exported_symbols() -> Tuple[str, ...]:
             "varlen_attn_launches_per_call", "varlen_attn_version",
             "varlen_attn_last_error_detail", "varlen_attn_fwd_noalloc", "varlen_attn_fwd_ex",
             "varlen_mask_to_seqlens", "varlen_gather_rows", "varlen_scatter_rows",
-            "varlen_fold_pair_bias_row", "varlen_attn_decode")
+            "varlen_fold_pair_bias_row", "varlen_attn_decode", "varlen_attn_bwd")
 
 
 def load_library():
@@ -88,6 +88,10 @@ def load_library():
     lib.varlen_attn_decode.argtypes = [vp, vp, i32, i32, i32, vp, vp, i32, vp, vp, vp, i32, i32,
                                        i32, f32, i32, i32, vp, vp, vp]
     lib.varlen_attn_decode.restype = i32
+    lib.varlen_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                    i32, i32, ctypes.c_float, i32, vp, vp, i64, i64, i64, i64,
+                                    ctypes.c_uint, vp, vp, vp, vp, vp, i64, i64, i64, vp]
+    lib.varlen_attn_bwd.restype = i32
     lib.varlen_attn_strerror.argtypes = [i32]
     lib.varlen_attn_strerror.restype = ctypes.c_char_p
     lib.varlen_attn_get_device_error.argtypes = [vp]
@@ -380,6 +384,84 @@ def fold_pair_bias_row(bias_pair, cu_seqlens_k, n_heads, total_k, row=0, head_di
             None if bias_in is None else _dev_ptr(bias_in), _dev_ptr(out),
             _stream_handle(stream)))
     return out
+
+
+def varlen_attn_bwd(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
+                    max_seqlen_k: int, softmax_scale: Optional[float] = None,
+                    causal: bool = False, bias_per_key=None, bias_pair=None,
+                    bias_pair_strides=None, bias_pair_kv_heads: bool = False,
+                    need_dbias_per_key: bool = False, need_dbias_pair: bool = False,
+                    dq=None, dk=None, dv=None, stream=None):
+    """Backward of ``varlen_attn_fwd`` (bf16) through the C ABI.
+
+    ``out`` and ``lse`` are the forward's results for the same arguments,
+    ``dout`` the gradient of the loss w.r.t. ``out``. Returns
+    ``(dq, dk, dv, dbias_per_key, dbias_pair)``: ``dq`` like q, ``dk``/``dv``
+    like k/v (bf16); ``dbias_per_key`` fp32 ``[total_k, n_heads]`` when
+    requested; ``dbias_pair`` fp32 ``[batch, n_heads, max_seqlen_q,
+    max_seqlen_k]`` per query head when requested (zeros outside the
+    sequences; sum over the heads that share a broadcast or per-K/V-head
+    grid for that grid's gradient). Unrequested ones are None.
+    """
+    import torch
+    lib = load_library()
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
+        if t.dim() != 3 or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 [tokens, heads, head_dim] tensor")
+    if out.shape != q.shape or dout.shape != q.shape or v.shape != k.shape:
+        raise ValueError("out and dout must have q's shape, v k's shape")
+    dev = q.device
+    tensors = [q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k] + \
+        [t for t in (bias_per_key, bias_pair, dq, dk, dv) if t is not None]
+    if dev.type != "cuda" or any(t.device != dev for t in tensors):
+        raise ValueError("all tensors must be on the same CUDA device")
+    if cu_seqlens_q.dtype != torch.int32 or cu_seqlens_k.dtype != torch.int32 or \
+            not cu_seqlens_q.is_contiguous() or not cu_seqlens_k.is_contiguous():
+        raise ValueError("cu_seqlens must be contiguous int32")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have batch + 1 entries")
+    total_q, n_heads, head_dim = q.shape
+    total_k, n_kv_heads, _ = k.shape
+    batch = cu_seqlens_q.numel() - 1
+    if lse.shape != (n_heads, total_q) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous fp32 [n_heads, total_q]")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(head_dim)
+    if bias_per_key is not None and (bias_per_key.dtype != torch.float32 or
+                                     not bias_per_key.is_contiguous() or
+                                     tuple(bias_per_key.shape) != (total_k, n_heads)):
+        raise ValueError("bias_per_key must be contiguous fp32 [total_k, n_heads]")
+    strides = (0, 0, 0, 0)
+    if bias_pair is not None:
+        if bias_pair.dtype != torch.float32:
+            raise ValueError("bias_pair must be fp32")
+        strides = _grid_strides(bias_pair, bias_pair_strides)
+    for name, t, ref in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
+        if t is not None and (t.shape != ref.shape or t.dtype != torch.bfloat16 or
+                              not t.is_contiguous()):
+            raise ValueError(f"{name} must be contiguous bf16 with the shape of its input")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    dbk = torch.empty((total_k, n_heads), dtype=torch.float32, device=dev) \
+        if need_dbias_per_key else None
+    dbp = None
+    dstr = (0, 0, 0)
+    if need_dbias_pair:
+        dbp = torch.zeros((batch, n_heads, max(int(max_seqlen_q), 1), max(int(max_seqlen_k), 1)),
+                          dtype=torch.float32, device=dev)
+        dstr = dbp.stride()[:3]
+    ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    flags = BIAS_PAIR_KV_HEADS if bias_pair_kv_heads else 0
+    with torch.cuda.device(dev):
+        status = lib.varlen_attn_bwd(
+            ptr(q), ptr(k), ptr(v), ptr(out), ptr(lse), ptr(dout), ptr(cu_seqlens_q),
+            ptr(cu_seqlens_k), batch, total_q, total_k, int(max_seqlen_q), int(max_seqlen_k),
+            n_heads, n_kv_heads, head_dim, float(softmax_scale), 1 if causal else 0,
+            ptr(bias_per_key), ptr(bias_pair), *strides, flags, ptr(dq), ptr(dk), ptr(dv),
+            ptr(dbk), ptr(dbp), *dstr, _stream_handle(stream))
+    _check(status)
+    return dq, dk, dv, dbk, dbp
 
 
 def varlen_attn_decode(q, cu_seqlens_q, max_seqlen_q: int, k_cache, v_cache, cache_seqlens,

@@ -1,0 +1,542 @@
+// Backward pass of packed variable-length attention for sm_100a.
+//
+// With P the forward's probabilities (recomputed from Q, K, the biases and
+// the forward's LSE), dO the output gradient and delta = rowsum(dO * O):
+//   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - delta),
+//   dQ = scale dS K,  dK = scale dS^T Q,  dbias_key = colsum(dS),  dbias_pair = dS
+// (the chain rule through the forward definition; the GiGL PR 858 page,
+// "Approach", notes that a varlen kernel with a per-sequence bias lacks this
+// backward, and the ASpec PR 25 page, "Verification", bounds Q/K/V gradient
+// errors at 1% relative L2 against a dense math backend).
+//
+// Two kernels, each deterministic (no atomics), one CTA per SM:
+//   attn_bwd_dkdv_sm100: one CTA per (sequence, K/V head, 128-key block).
+//     K and V stay in shared memory; for every query head of the group and
+//     every 128-row query block that can see the keys, Q and dO arrive by
+//     TMA (two stages) and the tensor cores compute
+//       S^T  = K Q^T       (tensor memory cols [0,128): keys are the lanes)
+//       dP^T = V dO^T      (cols [128,256))
+//     the four compute warps turn them into P^T and dS^T (bf16, written
+//     back over S^T and dP^T), and
+//       dV  += P^T dO      (cols [256, 256+D), P^T read from tensor memory)
+//       dK  += dS^T Q      (cols [256+D, 256+2D))
+//     Each thread owns one key, so the per-key bias gradient is a register
+//     sum and the pair-grid gradient rows are written coalesced.
+//   attn_bwd_dq_sm100: one CTA per (sequence, query head, 128-row block).
+//     Q and dO stay; K and V stream in two stages; S = Q K^T, dP = dO V^T,
+//     dS as above (one thread per query row), dQ += dS K.
+// The pair of kernels recomputes S and dP once more than a single fused
+// kernel with atomic dQ accumulation would; in exchange nothing is reduced
+// across CTAs and the results do not depend on scheduling.
+#pragma once
+#include "attn_sm100.cuh"
+
+namespace va {
+
+struct BwdParams {
+  const int* cu_q;
+  const int* cu_k;
+  const int* valid;               // 1 when the validation kernel accepted cu_seqlens
+  int total_q, total_k;
+  int n_heads, n_kv_heads, group;
+  int causal;
+  float scale;                    // softmax_scale
+  const float* lse;               // [Hq, Tq] natural log (forward output)
+  const float* delta;             // [Hq, Tq] rowsum(dO * O)
+  const float* bias_key;          // [Tk, Hq] or null
+  const float* bias_pair;         // strided grid or null
+  long long sb, sh, sr, sc;
+  int bias_head_div;
+  float* dbias_key;               // [Tk, Hq] or null
+  float* dbias_pair;              // [B, Hq, R, C] (column stride 1) or null
+  long long dsb, dsh, dsr;
+  void* dq;                       // bf16 [Tq, Hq, D]
+  void* dk;                       // bf16 [Tk, Hkv, D]
+  void* dv;                       // bf16 [Tk, Hkv, D]
+  int* error;
+};
+
+constexpr int kBwdThreads = 192;  // compute warps 0-3, MMA warp 4, load warp 5
+constexpr int kBwdMmaWarp = 4;
+constexpr int kBwdLoadWarp = 5;
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kChunk = 128 * 128;               // 128 rows x 64 bf16 (128 B)
+  static constexpr int kTile = (D / 64) * kChunk;         // 128 rows x D bf16
+  static constexpr int kFixedOff = 0;                     // two resident tiles
+  static constexpr int kStageOff = 2 * kTile;             // two stages of two tiles
+  static constexpr int kRowOff = kStageOff + 4 * kTile;   // float [2 buf][2][128]
+  static constexpr int kBarOff = kRowOff + 2 * 2 * 128 * 4;
+  // fixed_full, st_full[2], st_empty[2], s_full, p_full, o_full, rows_full[2]
+  static constexpr int kNumBars = 10;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem slot, abort flag
+  static constexpr int kUsed = kMiscOff + 16 + 1024;       // + alignment slack
+  // At least 120 KB so that one CTA (holding all 512 tensor-memory columns)
+  // runs per SM.
+  static constexpr int kSmemBytes = kUsed < 120 * 1024 ? 120 * 1024 : kUsed;
+};
+
+template <int D>
+struct BwdSmem {
+  uint8_t* base;
+  __device__ uint8_t* fixed(int i) const { return base + BwdCfg<D>::kFixedOff + i * BwdCfg<D>::kTile; }
+  __device__ uint8_t* stage(int st, int i) const {
+    return base + BwdCfg<D>::kStageOff + (2 * st + i) * BwdCfg<D>::kTile;
+  }
+  __device__ float* rows(int b, int i) const {
+    return reinterpret_cast<float*>(base + BwdCfg<D>::kRowOff) + (2 * b + i) * 128;
+  }
+  __device__ uint64_t* bars() const { return reinterpret_cast<uint64_t*>(base + BwdCfg<D>::kBarOff); }
+  __device__ uint64_t* fixed_full() const { return bars(); }
+  __device__ uint64_t* st_full(int st) const { return bars() + 1 + st; }
+  __device__ uint64_t* st_empty(int st) const { return bars() + 3 + st; }
+  __device__ uint64_t* s_full() const { return bars() + 5; }
+  __device__ uint64_t* p_full() const { return bars() + 6; }
+  __device__ uint64_t* o_full() const { return bars() + 7; }
+  __device__ uint64_t* rows_full(int b) const { return bars() + 8 + b; }
+  __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + BwdCfg<D>::kMiscOff); }
+  __device__ int* abort_flag() const { return reinterpret_cast<int*>(base + BwdCfg<D>::kMiscOff + 4); }
+};
+
+// delta[h, t] = sum_d dO[t, h, d] * O[t, h, d] (fp32 from bf16), one thread
+// per (token, head), 16-byte loads.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_delta_kernel(const __nv_bfloat16* __restrict__ out,
+                                                        const __nv_bfloat16* __restrict__ dout,
+                                                        int total_q, int n_heads,
+                                                        float* __restrict__ delta) {
+  const long long n = (long long)total_q * n_heads;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const uint4* o = reinterpret_cast<const uint4*>(out + i * D);
+    const uint4* g = reinterpret_cast<const uint4*>(dout + i * D);
+    float acc = 0.f;
+#pragma unroll 4
+    for (int u = 0; u < D / 8; ++u) {
+      const uint4 a = __ldg(o + u), b = __ldg(g + u);
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc = fmaf(__uint_as_float(av[e] << 16), __uint_as_float(bv[e] << 16), acc);
+        acc = fmaf(__uint_as_float(av[e] & 0xffff0000u), __uint_as_float(bv[e] & 0xffff0000u), acc);
+      }
+    }
+    const long long t = i / n_heads, h = i % n_heads;
+    delta[h * total_q + t] = acc;
+  }
+}
+
+// Shared setup of both kernels: barriers, tensor memory, smem base.
+template <int D>
+__device__ __forceinline__ uint32_t bwd_setup(BwdSmem<D>& sm, uint8_t* smem_raw) {
+  {
+    const uint32_t a = ptx::smem_u32(smem_raw);
+    sm.base = smem_raw + ((1024 - (a & 1023)) & 1023);
+  }
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(sm.fixed_full(), 1);
+    for (int st = 0; st < 2; ++st) {
+      ptx::mbar_init(sm.st_full(st), 1);
+      ptx::mbar_init(sm.st_empty(st), 1);
+    }
+    ptx::mbar_init(sm.s_full(), 1);
+    ptx::mbar_init(sm.p_full(), 128);
+    ptx::mbar_init(sm.o_full(), 1);
+    ptx::mbar_init(sm.rows_full(0), 128);
+    ptx::mbar_init(sm.rows_full(1), 128);
+    *sm.abort_flag() = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == kBwdMmaWarp) {
+    ptx::tmem_alloc(sm.tmem_slot(), 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  return *sm.tmem_slot();
+}
+
+template <int D>
+__device__ __forceinline__ void bwd_teardown(const BwdSmem<D>& sm, uint32_t tmem) {
+  ptx::tc_fence_before();
+  __syncthreads();
+  if ((threadIdx.x >> 5) == kBwdMmaWarp) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
+// Loads a 128-row x D tile (D/64 swizzled chunks) at (head, row).
+template <int D>
+__device__ __forceinline__ void bwd_load_tile(uint8_t* dst, const CUtensorMap* tm, uint64_t* bar,
+                                              int head, int row) {
+#pragma unroll
+  for (int c = 0; c < D / 64; ++c)
+    ptx::tma_load_3d(dst + c * BwdCfg<D>::kChunk, tm, bar, c * 64, head, row);
+}
+
+// Accumulator rows of tensor memory (D fp32 columns at `t`) -> bf16 row of
+// `dst` times `mul`, or zeros when `have` is false.
+template <int D>
+__device__ __forceinline__ void bwd_store_row(uint32_t t, bool have, float mul, __nv_bfloat16* dst,
+                                              bool ok) {
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t v[32];
+    if (have) {
+      ptx::tmem_ld32(t + c * 32, v);
+      ptx::tmem_wait_ld();
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = 0u;
+    }
+    if (ok) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        uint4 w;
+        w.x = ptx::pack_bf16x2(__uint_as_float(v[8 * u + 0]) * mul, __uint_as_float(v[8 * u + 1]) * mul);
+        w.y = ptx::pack_bf16x2(__uint_as_float(v[8 * u + 2]) * mul, __uint_as_float(v[8 * u + 3]) * mul);
+        w.z = ptx::pack_bf16x2(__uint_as_float(v[8 * u + 4]) * mul, __uint_as_float(v[8 * u + 5]) * mul);
+        w.w = ptx::pack_bf16x2(__uint_as_float(v[8 * u + 6]) * mul, __uint_as_float(v[8 * u + 7]) * mul);
+        d4[u] = w;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ dK, dV
+template <int D, bool kBiasKey, bool kBiasPair>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const unsigned FULL = 0xffffffffu;
+  const int kb = blockIdx.x, kvh = blockIdx.y, seq = blockIdx.z;
+  const int q0 = p.cu_q[seq], k0 = p.cu_k[seq];
+  const int Lq = p.cu_q[seq + 1] - q0, Lk = p.cu_k[seq + 1] - k0;
+  if (*p.valid == 0 || kb * BN >= Lk) return;  // uniform over the CTA, before any barrier
+  const int off = Lk - Lq;    // bottom-right causal offset
+  int qb0 = 0;
+  if (p.causal) {
+    const int qmin = kb * BN - off;  // first query row that sees key kb*BN
+    qb0 = qmin > 0 ? qmin / BM : 0;
+  }
+  const int nqb = ceil_div(Lq, BM);
+  const int per_head = nqb > qb0 ? nqb - qb0 : 0;
+  const int G = p.group;
+  const int n_tiles = per_head * G;
+
+  BwdSmem<D> sm;
+  const uint32_t tmem = bwd_setup<D>(sm, smem_raw);
+  const Ctl ctl{sm.abort_flag(), p.error};
+  const int warp = threadIdx.x >> 5;
+
+  if (warp == kBwdLoadWarp) {
+    int uses[2] = {0, 0};
+    bool ok = true;
+    if (ptx::elect_one()) {
+      ptx::mbar_arrive_expect_tx(sm.fixed_full(), 2 * BwdCfg<D>::kTile);
+      bwd_load_tile<D>(sm.fixed(0), &tm_k, sm.fixed_full(), kvh, k0 + kb * BN);
+      bwd_load_tile<D>(sm.fixed(1), &tm_v, sm.fixed_full(), kvh, k0 + kb * BN);
+    }
+    __syncwarp();
+    for (int t = 0; t < n_tiles && ok; ++t) {
+      const int st = t & 1;
+      ok = __all_sync(FULL, wait_bar(sm.st_empty(st), ((t >> 1) & 1) ^ 1, ctl));
+      if (!ok) break;
+      ++uses[st];
+      const int h = kvh * G + t / per_head;
+      const int row = q0 + (qb0 + t % per_head) * BM;
+      if (ptx::elect_one()) {
+        ptx::mbar_arrive_expect_tx(sm.st_full(st), 2 * BwdCfg<D>::kTile);
+        bwd_load_tile<D>(sm.stage(st, 0), &tm_q, sm.st_full(st), h, row);
+        bwd_load_tile<D>(sm.stage(st, 1), &tm_do, sm.st_full(st), h, row);
+      }
+      __syncwarp();
+    }
+    drain_bar(sm.fixed_full(), 0);
+    for (int st = 0; st < 2; ++st)
+      if (uses[st] > 0) drain_bar(sm.st_full(st), (uses[st] - 1) & 1);
+  } else if (warp == kBwdMmaWarp) {
+    const uint64_t kd = desc_kmajor_sw128(ptx::smem_u32(sm.fixed(0)));
+    const uint64_t vd = desc_kmajor_sw128(ptx::smem_u32(sm.fixed(1)));
+    bool ok = __all_sync(FULL, wait_bar(sm.fixed_full(), 0, ctl));
+    for (int t = 0; t < n_tiles && ok; ++t) {
+      const int st = t & 1;
+      ok = __all_sync(FULL, wait_bar(sm.st_full(st), (t >> 1) & 1, ctl));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      const uint32_t qa = ptx::smem_u32(sm.stage(st, 0)), da = ptx::smem_u32(sm.stage(st, 1));
+      if (ptx::elect_one()) {
+        issue_s<D>(tmem + 0, kd, desc_kmajor_sw128(qa));     // S^T  = K Q^T
+        issue_s<D>(tmem + 128, vd, desc_kmajor_sw128(da));   // dP^T = V dO^T
+        ptx::tc_commit(sm.s_full());
+      }
+      __syncwarp();
+      ok = __all_sync(FULL, wait_bar(sm.p_full(), t & 1, ctl));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      if (ptx::elect_one()) {
+        const uint64_t dmn = desc_mnmajor_sw128(da, BwdCfg<D>::kChunk);
+        const uint64_t qmn = desc_mnmajor_sw128(qa, BwdCfg<D>::kChunk);
+        issue_pv_half<D>(tmem + 256, tmem + 0, dmn, 0, t > 0);       // dV += P^T dO
+        issue_pv_half<D>(tmem + 256, tmem + 0, dmn, 1, true);
+        issue_pv_half<D>(tmem + 256 + D, tmem + 128, qmn, 0, t > 0); // dK += dS^T Q
+        issue_pv_half<D>(tmem + 256 + D, tmem + 128, qmn, 1, true);
+        ptx::tc_commit(sm.st_empty(st));
+      }
+      __syncwarp();
+    }
+    if (ptx::elect_one()) ptx::tc_commit(sm.o_full());
+    __syncwarp();
+    drain_bar(sm.o_full(), 0);
+  } else {
+    // compute warps: thread c owns key kb*BN + c (tensor-memory lane c)
+    const int c = threadIdx.x;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t t_s = tmem + lane_base, t_dp = tmem + lane_base + 128;
+    const int kc = kb * BN + c;
+    const bool key_ok = kc < Lk;
+    const float kL2 = kLog2e;
+    float dbk = 0.f, bkey = 0.f;
+    bool ok = true;
+    for (int t = 0; t < n_tiles && ok; ++t) {
+      const int g = t / per_head, qb = qb0 + t % per_head;
+      const int h = kvh * G + g;
+      if (t % per_head == 0) {
+        dbk = 0.f;
+        if constexpr (kBiasKey) bkey = key_ok ? p.bias_key[(long long)(k0 + kc) * p.n_heads + h] : 0.f;
+      }
+      // this tile's row constants: LSE * log2(e) and delta
+      {
+        const int b = t & 1;
+        const int rl = qb * BM + c;
+        const long long gi = (long long)h * p.total_q + q0 + rl;
+        sm.rows(b, 0)[c] = rl < Lq ? p.lse[gi] * kL2 : 0.f;
+        sm.rows(b, 1)[c] = rl < Lq ? p.delta[gi] : 0.f;
+        // Buffer b is written again at tile t + 2, after every thread has
+        // arrived for tile t + 1, i.e. finished reading it for tile t.
+        ptx::mbar_arrive(sm.rows_full(b));
+        ok = __all_sync(FULL, wait_bar(sm.rows_full(b), (t >> 1) & 1, ctl));
+        if (!ok) break;
+      }
+      const float* lse2 = sm.rows(t & 1, 0);
+      const float* dl = sm.rows(t & 1, 1);
+      ok = __all_sync(FULL, wait_bar(sm.s_full(), t & 1, ctl));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      const float* grow = nullptr;
+      if constexpr (kBiasPair)
+        grow = p.bias_pair + (long long)seq * p.sb + (long long)(h / p.bias_head_div) * p.sh +
+               (long long)kc * p.sc;
+      float* dgrow = p.dbias_pair == nullptr
+                         ? nullptr
+                         : p.dbias_pair + (long long)seq * p.dsb + (long long)h * p.dsh + kc;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t s[32], dp[32];
+        ptx::tmem_ld32(t_s + cc * 32, s);
+        ptx::tmem_ld32(t_dp + cc * 32, dp);
+        ptx::tmem_wait_ld();
+        uint32_t pk[16], dk16[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float pv[2], dsv[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int r = cc * 32 + e + u;
+            const int ql = qb * BM + r;
+            const bool in = key_ok && ql < Lq;
+            const bool vis = in && (!p.causal || kc <= ql + off);
+            float x = __uint_as_float(s[e + u]) * p.scale;
+            if constexpr (kBiasKey) x += bkey;
+            if constexpr (kBiasPair) {
+              if (vis) x += __ldg(grow + (long long)ql * p.sr);
+            }
+            const float pr = vis ? ptx::ex2(fmaf(x, kL2, -lse2[r])) : 0.f;
+            const float ds = pr * (__uint_as_float(dp[e + u]) - dl[r]);
+            dbk += ds;
+            if (dgrow != nullptr && in) dgrow[(long long)ql * p.dsr] = ds;
+            pv[u] = pr;
+            dsv[u] = ds;
+          }
+          pk[e / 2] = ptx::pack_bf16x2(pv[0], pv[1]);
+          dk16[e / 2] = ptx::pack_bf16x2(dsv[0], dsv[1]);
+        }
+        // P^T over S^T and dS^T over dP^T: chunk cc only covers columns
+        // [16cc, 16cc + 16), which were read in this or an earlier chunk.
+        ptx::tmem_st16(t_s + cc * 16, pk);
+        ptx::tmem_st16(t_dp + cc * 16, dk16);
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(sm.p_full());
+      if (p.dbias_key != nullptr && key_ok && t % per_head == per_head - 1)
+        p.dbias_key[(long long)(k0 + kc) * p.n_heads + h] = dbk;
+    }
+    if (ok && p.dbias_key != nullptr && key_ok && per_head == 0)
+      for (int g = 0; g < G; ++g) p.dbias_key[(long long)(k0 + kc) * p.n_heads + kvh * G + g] = 0.f;
+    const bool have = n_tiles > 0;
+    if (have) {
+      ok = ok && __all_sync(FULL, wait_bar(sm.o_full(), 0, ctl));
+      ptx::tc_fence_after();
+    }
+    if (ok) {
+      const long long o = ((long long)(k0 + kc) * p.n_kv_heads + kvh) * D;
+      bwd_store_row<D>(tmem + lane_base + 256, have, 1.f,
+                       reinterpret_cast<__nv_bfloat16*>(p.dv) + o, key_ok);
+      bwd_store_row<D>(tmem + lane_base + 256 + D, have, p.scale,
+                       reinterpret_cast<__nv_bfloat16*>(p.dk) + o, key_ok);
+    }
+  }
+  bwd_teardown<D>(sm, tmem);
+}
+
+// ------------------------------------------------------------------ dQ
+template <int D, bool kBiasKey, bool kBiasPair>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dq_sm100(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const unsigned FULL = 0xffffffffu;
+  const int qb = blockIdx.x, h = blockIdx.y, seq = blockIdx.z;
+  const int q0 = p.cu_q[seq], k0 = p.cu_k[seq];
+  const int Lq = p.cu_q[seq + 1] - q0, Lk = p.cu_k[seq + 1] - k0;
+  if (*p.valid == 0 || qb * BM >= Lq) return;  // uniform over the CTA, before any barrier
+  const int off = Lk - Lq;
+  const int rows = min(BM, Lq - qb * BM);
+  const int n_k = slot_tiles(qb * BM, rows, Lq, Lk, p.causal);
+  const int kvh = h / p.group;
+
+  BwdSmem<D> sm;
+  const uint32_t tmem = bwd_setup<D>(sm, smem_raw);
+  const Ctl ctl{sm.abort_flag(), p.error};
+  const int warp = threadIdx.x >> 5;
+
+  if (warp == kBwdLoadWarp) {
+    int uses[2] = {0, 0};
+    bool ok = true;
+    if (n_k > 0 && ptx::elect_one()) {
+      ptx::mbar_arrive_expect_tx(sm.fixed_full(), 2 * BwdCfg<D>::kTile);
+      bwd_load_tile<D>(sm.fixed(0), &tm_q, sm.fixed_full(), h, q0 + qb * BM);
+      bwd_load_tile<D>(sm.fixed(1), &tm_do, sm.fixed_full(), h, q0 + qb * BM);
+    }
+    __syncwarp();
+    for (int j = 0; j < n_k && ok; ++j) {
+      const int st = j & 1;
+      ok = __all_sync(FULL, wait_bar(sm.st_empty(st), ((j >> 1) & 1) ^ 1, ctl));
+      if (!ok) break;
+      ++uses[st];
+      if (ptx::elect_one()) {
+        ptx::mbar_arrive_expect_tx(sm.st_full(st), 2 * BwdCfg<D>::kTile);
+        bwd_load_tile<D>(sm.stage(st, 0), &tm_k, sm.st_full(st), kvh, k0 + j * BN);
+        bwd_load_tile<D>(sm.stage(st, 1), &tm_v, sm.st_full(st), kvh, k0 + j * BN);
+      }
+      __syncwarp();
+    }
+    if (n_k > 0) drain_bar(sm.fixed_full(), 0);
+    for (int st = 0; st < 2; ++st)
+      if (uses[st] > 0) drain_bar(sm.st_full(st), (uses[st] - 1) & 1);
+  } else if (warp == kBwdMmaWarp) {
+    const uint64_t qd = desc_kmajor_sw128(ptx::smem_u32(sm.fixed(0)));
+    const uint64_t dod = desc_kmajor_sw128(ptx::smem_u32(sm.fixed(1)));
+    bool ok = n_k == 0 || __all_sync(FULL, wait_bar(sm.fixed_full(), 0, ctl));
+    for (int j = 0; j < n_k && ok; ++j) {
+      const int st = j & 1;
+      ok = __all_sync(FULL, wait_bar(sm.st_full(st), (j >> 1) & 1, ctl));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      const uint32_t ka = ptx::smem_u32(sm.stage(st, 0)), va_ = ptx::smem_u32(sm.stage(st, 1));
+      if (ptx::elect_one()) {
+        issue_s<D>(tmem + 0, qd, desc_kmajor_sw128(ka));      // S  = Q K^T
+        issue_s<D>(tmem + 128, dod, desc_kmajor_sw128(va_));  // dP = dO V^T
+        ptx::tc_commit(sm.s_full());
+      }
+      __syncwarp();
+      ok = __all_sync(FULL, wait_bar(sm.p_full(), j & 1, ctl));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      if (ptx::elect_one()) {
+        const uint64_t kmn = desc_mnmajor_sw128(ka, BwdCfg<D>::kChunk);
+        issue_pv_half<D>(tmem + 256, tmem + 128, kmn, 0, j > 0);  // dQ += dS K
+        issue_pv_half<D>(tmem + 256, tmem + 128, kmn, 1, true);
+        ptx::tc_commit(sm.st_empty(st));
+      }
+      __syncwarp();
+    }
+    if (ptx::elect_one()) ptx::tc_commit(sm.o_full());
+    __syncwarp();
+    drain_bar(sm.o_full(), 0);
+  } else {
+    // compute warps: thread r owns query row qb*BM + r
+    const int r = threadIdx.x;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t t_s = tmem + lane_base, t_dp = tmem + lane_base + 128;
+    const int ql = qb * BM + r;
+    const bool row_ok = ql < Lq;
+    const long long gi = (long long)h * p.total_q + q0 + ql;
+    const float lse2 = row_ok ? p.lse[gi] * kLog2e : 0.f;
+    const float dl = row_ok ? p.delta[gi] : 0.f;
+    const float* grow = nullptr;
+    if constexpr (kBiasPair)
+      grow = p.bias_pair + (long long)seq * p.sb + (long long)(h / p.bias_head_div) * p.sh +
+             (long long)ql * p.sr;
+    bool ok = true;
+    for (int j = 0; j < n_k && ok; ++j) {
+      ok = __all_sync(FULL, wait_bar(sm.s_full(), j & 1, ctl));
+      if (!ok) break;
+      ptx::tc_fence_after();
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t s[32], dp[32];
+        ptx::tmem_ld32(t_s + cc * 32, s);
+        ptx::tmem_ld32(t_dp + cc * 32, dp);
+        ptx::tmem_wait_ld();
+        uint32_t dk16[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float dsv[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int kc = j * BN + cc * 32 + e + u;
+            const bool vis = row_ok && kc < Lk && (!p.causal || kc <= ql + off);
+            float x = __uint_as_float(s[e + u]) * p.scale;
+            if constexpr (kBiasKey) {
+              if (vis) x += __ldg(p.bias_key + (long long)(k0 + kc) * p.n_heads + h);
+            }
+            if constexpr (kBiasPair) {
+              if (vis) x += __ldg(grow + (long long)kc * p.sc);
+            }
+            const float pr = vis ? ptx::ex2(fmaf(x, kLog2e, -lse2)) : 0.f;
+            dsv[u] = pr * (__uint_as_float(dp[e + u]) - dl);
+          }
+          dk16[e / 2] = ptx::pack_bf16x2(dsv[0], dsv[1]);
+        }
+        ptx::tmem_st16(t_dp + cc * 16, dk16);
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(sm.p_full());
+    }
+    const bool have = n_k > 0;
+    if (have) {
+      ok = ok && __all_sync(FULL, wait_bar(sm.o_full(), 0, ctl));
+      ptx::tc_fence_after();
+    }
+    if (ok)
+      bwd_store_row<D>(tmem + lane_base + 256, have, p.scale,
+                       reinterpret_cast<__nv_bfloat16*>(p.dq) + ((long long)(q0 + ql) * p.n_heads + h) * D,
+                       row_ok);
+  }
+  bwd_teardown<D>(sm, tmem);
+}
+
+}  // namespace va

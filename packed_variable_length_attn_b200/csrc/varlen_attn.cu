@@ -19,6 +19,7 @@
 #include "sched.cuh"
 #include "layout.cuh"
 #include "decode.cuh"
+#include "bwd_sm100.cuh"
 
 // ---------------------------------------------------------------------------
 // Fixed scratch for varlen_attn_fwd_noalloc.
@@ -391,6 +392,27 @@ int launch_decode(dim3 grid, const DecodeParams& dp, cudaStream_t st) {
 }
 
 }  // namespace
+
+template <int D, bool BK, bool BP>
+int launch_bwd(dim3 grid_a, dim3 grid_q, const CUtensorMap& tq, const CUtensorMap& tk,
+               const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& bp,
+               cudaStream_t st) {
+  auto ka = attn_bwd_dkdv_sm100<D, BK, BP>;
+  auto kq = attn_bwd_dq_sm100<D, BK, BP>;
+  static thread_local int configured_for = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_for != dev) {
+    int rc;
+    if ((rc = set_smem(ka, BwdCfg<D>::kSmemBytes)) || (rc = set_smem(kq, BwdCfg<D>::kSmemBytes)))
+      return rc;
+    configured_for = dev;
+  }
+  ka<<<grid_a, kBwdThreads, BwdCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, bp);
+  if (int rc = check_launch("attn_bwd_dkdv_sm100")) return rc;
+  kq<<<grid_q, kBwdThreads, BwdCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, bp);
+  return check_launch("attn_bwd_dq_sm100");
+}
 
 extern "C" {
 
@@ -824,6 +846,125 @@ int varlen_attn_set_profile_events(void* start_event, void* stop_event) {
   t_ev_start = static_cast<cudaEvent_t>(start_event);
   t_ev_stop = static_cast<cudaEvent_t>(stop_event);
   return VARLEN_ATTN_OK;
+}
+
+int varlen_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                    const float* lse, const void* dout, const int32_t* cu_seqlens_q,
+                    const int32_t* cu_seqlens_k, int batch, int total_q, int total_k,
+                    int max_seqlen_q, int max_seqlen_k, int n_heads, int n_kv_heads,
+                    int head_dim, float softmax_scale, int causal, const float* bias_per_key,
+                    const float* bias_pair, int64_t bias_stride_b, int64_t bias_stride_h,
+                    int64_t bias_stride_q, int64_t bias_stride_k, unsigned flags, void* dq,
+                    void* dk, void* dv, float* dbias_per_key, float* dbias_pair,
+                    int64_t dbias_stride_b, int64_t dbias_stride_h, int64_t dbias_stride_q,
+                    void* stream) {
+  if (flags & ~(unsigned)VARLEN_ATTN_BIAS_PAIR_KV_HEADS) return VARLEN_ATTN_ERR_BAD_BIAS;
+  Common a{batch, total_q, total_k, max_seqlen_q, max_seqlen_k, n_heads, n_kv_heads, head_dim,
+           causal ? 1 : 0, cu_seqlens_q, cu_seqlens_k, bias_per_key, bias_pair, bias_stride_b,
+           bias_stride_h, bias_stride_q, bias_stride_k};
+  int rc = validate_common(a, q, k, v, out, lse);
+  if (rc) return rc;
+  if (!lse || !dout || !dq || !dk || !dv) return VARLEN_ATTN_ERR_NULL_POINTER;
+  if (!aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      (dbias_per_key && !aligned(dbias_per_key, 4)) || (dbias_pair && !aligned(dbias_pair, 4)))
+    return VARLEN_ATTN_ERR_MISALIGNED;
+  if (dbias_pair && (dbias_stride_b < 0 || dbias_stride_h < 0 || dbias_stride_q < 0))
+    return VARLEN_ATTN_ERR_BAD_BIAS;
+  if (batch > 65535 || n_heads > 65535) return VARLEN_ATTN_ERR_TOO_LARGE;
+  DeviceInfo* di = nullptr;
+  if ((rc = device_info(&di))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (total_q == 0 && total_k == 0) return VARLEN_ATTN_OK;
+
+  // workspace: schedule header (validation result) + delta [Hq, Tq]
+  void* wsp = nullptr;
+  const size_t delta_bytes = (size_t)n_heads * (size_t)(total_q > 0 ? total_q : 1) * 4;
+  if ((rc = workspace(stream, 256 + 2 * sizeof(int2) + delta_bytes, &wsp))) return rc;
+  Workspace ws = carve(wsp, 1);
+  float* delta = reinterpret_cast<float*>(static_cast<char*>(wsp) + 256 + 2 * sizeof(int2));
+
+  SchedParams sp;
+  sp.cu_q = cu_seqlens_q;
+  sp.cu_k = cu_seqlens_k;
+  sp.batch = batch;
+  sp.total_q = total_q;
+  sp.total_k = total_k;
+  sp.max_q = max_seqlen_q;
+  sp.max_k = max_seqlen_k;
+  sp.causal = a.causal;
+  sp.pairing = -1;  // validate only: count = 1 when the boundaries are sound, else 0
+  sp.n_hg = 1;
+  sp.ws = ws;
+  sp.error = di->error_word;
+  if ((rc = launch_schedule(sp, st))) return rc;
+
+  if (total_q > 0) {
+    const long long n = (long long)total_q * n_heads;
+    const int blocks = (int)std::min<long long>((n + 255) / 256, (long long)di->sm_count * 8);
+    if (head_dim == 64)
+      bwd_delta_kernel<64><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(out),
+                                                   static_cast<const __nv_bfloat16*>(dout),
+                                                   total_q, n_heads, delta);
+    else
+      bwd_delta_kernel<128><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(out),
+                                                    static_cast<const __nv_bfloat16*>(dout),
+                                                    total_q, n_heads, delta);
+    if ((rc = check_launch("bwd_delta_kernel"))) return rc;
+  }
+
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_tmap(&tq, q, head_dim, n_heads, total_q, BM) ||
+      !make_tmap(&tdo, dout, head_dim, n_heads, total_q, BM) ||
+      !make_tmap(&tk, k, head_dim, n_kv_heads, total_k, BN) ||
+      !make_tmap(&tv, v, head_dim, n_kv_heads, total_k, BN))
+    return VARLEN_ATTN_ERR_CUDA;
+
+  BwdParams bp;
+  bp.cu_q = cu_seqlens_q;
+  bp.cu_k = cu_seqlens_k;
+  bp.valid = ws.count;
+  bp.total_q = total_q;
+  bp.total_k = total_k;
+  bp.n_heads = n_heads;
+  bp.n_kv_heads = n_kv_heads;
+  bp.group = n_heads / n_kv_heads;
+  bp.causal = a.causal;
+  bp.scale = softmax_scale;
+  bp.lse = lse;
+  bp.delta = delta;
+  bp.bias_key = bias_per_key;
+  bp.bias_pair = bias_pair;
+  bp.sb = bias_stride_b;
+  bp.sh = bias_stride_h;
+  bp.sr = bias_stride_q;
+  bp.sc = bias_stride_k;
+  bp.bias_head_div = (flags & VARLEN_ATTN_BIAS_PAIR_KV_HEADS) ? bp.group : 1;
+  bp.dbias_key = dbias_per_key;
+  bp.dbias_pair = dbias_pair;
+  bp.dsb = dbias_stride_b;
+  bp.dsh = dbias_stride_h;
+  bp.dsr = dbias_stride_q;
+  bp.dq = dq;
+  bp.dk = dk;
+  bp.dv = dv;
+  bp.error = di->error_word;
+  const dim3 grid_a((unsigned)std::max(1, ceil_div(max_seqlen_k, BN)), (unsigned)n_kv_heads,
+                    (unsigned)batch);
+  const dim3 grid_q((unsigned)std::max(1, ceil_div(max_seqlen_q, BM)), (unsigned)n_heads,
+                    (unsigned)batch);
+  const bool bk = bias_per_key != nullptr, bpr = bias_pair != nullptr;
+  if (head_dim == 64) {
+    if (bk && bpr) rc = launch_bwd<64, true, true>(grid_a, grid_q, tq, tk, tv, tdo, bp, st);
+    else if (bk) rc = launch_bwd<64, true, false>(grid_a, grid_q, tq, tk, tv, tdo, bp, st);
+    else if (bpr) rc = launch_bwd<64, false, true>(grid_a, grid_q, tq, tk, tv, tdo, bp, st);
+    else rc = launch_bwd<64, false, false>(grid_a, grid_q, tq, tk, tv, tdo, bp, st);
+  } else {
+    if (bk && bpr) rc = launch_bwd<128, true, true>(grid_a, grid_q, tq, tk, tv, tdo, bp, st);
+    else if (bk) rc = launch_bwd<128, true, false>(grid_a, grid_q, tq, tk, tv, tdo, bp, st);
+    else if (bpr) rc = launch_bwd<128, false, true>(grid_a, grid_q, tq, tk, tv, tdo, bp, st);
+    else rc = launch_bwd<128, false, false>(grid_a, grid_q, tq, tk, tv, tdo, bp, st);
+  }
+  return rc;
 }
 
 int varlen_attn_launches_per_call(int fp32_path) {

@@ -136,3 +136,30 @@ def test_decode_host_validation_codes(lib):
     assert call(d=96) == 4
     assert call(mq=9, hq=8, hkv=2) == 2   # 9 x G=4 > 32 rows: the packed forward's job
     assert call(kc=24) == 5
+
+
+def test_backward_host_validation_codes(lib):
+    p = ctypes.c_void_p
+
+    def call(**kw):
+        a = dict(q=16, k=16, v=16, out=16, lse=16, dout=16, cuq=16, cuk=16, batch=2, tq=4, tk=4,
+                 mq=2, mk=2, hq=4, hkv=2, d=64, scale=0.1, causal=1, bk=None, bp=None,
+                 flags=0, dq=16, dk=16, dv=16, dbk=None, dbp=None, dsb=0)
+        a.update(kw)
+        q_ = lambda x: None if x is None else p(x)
+        return lib.varlen_attn_bwd(
+            q_(a["q"]), q_(a["k"]), q_(a["v"]), q_(a["out"]), q_(a["lse"]), q_(a["dout"]),
+            q_(a["cuq"]), q_(a["cuk"]), a["batch"], a["tq"], a["tk"], a["mq"], a["mk"], a["hq"],
+            a["hkv"], a["d"], a["scale"], a["causal"], q_(a["bk"]), q_(a["bp"]), 0, 0, 0, 0,
+            a["flags"], q_(a["dq"]), q_(a["dk"]), q_(a["dv"]), q_(a["dbk"]), q_(a["dbp"]),
+            a["dsb"], 0, 0, None)
+    assert call(lse=None) == 1
+    assert call(dout=None) == 1
+    assert call(dk=None) == 1
+    assert call(batch=0) == 2
+    assert call(hq=6, hkv=4) == 3
+    assert call(d=96) == 4
+    assert call(dq=24) == 5
+    assert call(dbp=16, dsb=-1) == 6
+    assert call(flags=2) == 6
+    assert call(batch=70000) == 11
