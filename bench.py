@@ -587,6 +587,72 @@ def run_decode(args, world, rank, local):
                      "peak_source": f"{src} hbm_gbs"}}), flush=True)
 
 
+def run_backward(args, world, rank, local):
+    """Backward pass of the named workload (default: the long causal GQA
+    batch): dQ, dK, dV (and the bias gradients where the workload has biases)
+    from the forward's output and LSE and a seeded dO. Useful FLOPs = 2.5x the
+    forward's (five products of 2*D per visible pair and head: S, dP, dV, dK,
+    dQ); the kernels' own recomputation of S and dP for dQ is not counted."""
+    import torch
+    import packed_variable_length_attn_b200 as va
+    from packed_variable_length_attn_b200 import metrics
+    if rank != 0:
+        return
+    torch.cuda.set_device(local)
+    w = _workload(args)
+    dev = torch.device("cuda", local)
+    q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
+    cu_q, cu_k = w.cu_q.to(dev), w.cu_k.to(dev)
+    bk = None if w.bias_key is None else w.bias_key.to(dev)
+    bp = None if w.bias_pair is None else w.bias_pair.to(dev)
+    kw = dict(softmax_scale=w.softmax_scale, causal=w.causal, bias_per_key=bk, bias_pair=bp,
+              bias_pair_strides=w.bias_strides if bp is not None else None)
+    out, lse = va.varlen_attn_fwd(q, k, v, cu_q, cu_k, w.max_seqlen_q, w.max_seqlen_k, **kw)
+    g = torch.Generator("cpu").manual_seed(20261301)
+    dout = torch.randn(w.q.shape, generator=g).to(torch.bfloat16).to(dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def step():
+        va.varlen_attn_bwd(q, k, v, out, lse, dout, cu_q, cu_k, w.max_seqlen_q, w.max_seqlen_k,
+                           need_dbias_per_key=bk is not None, need_dbias_pair=bp is not None,
+                           dq=dq, dk=dk, dv=dv, **kw)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    clocks.stop()
+    clk = clocks.summary()
+    ms = t0.elapsed_time(t1) / args.steps
+    if va.get_device_error() != 0:
+        raise RuntimeError("device error in the backward pass")
+    fwd_flops = metrics.useful_flops(w.lengths_q, w.lengths_k, w.causal, w.n_heads, w.head_dim)
+    flops = 2.5 * fwd_flops
+    tf = flops / (ms * 1e-3) / 1e12
+    peaks, src = _peaks()
+    peak = float(peaks["bf16_tflops"])
+    cfg = _config(w, args)
+    cfg["pass"] = "backward (dQ, dK, dV" + (", bias gradients)" if bk is not None or
+                                            bp is not None else ")")
+    print(json.dumps({
+        "metric": "varlen attn bwd useful TFLOP/s on 1 B200", "value": tf, "unit": "TFLOP/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 Q/K/V/dO)", "config": cfg,
+        "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tf / peak, "traffic": None, "peak_source": f"{src} bf16_tflops",
+                     "useful_flops_per_step": flops},
+        "gpu_launches": 4 * args.steps, "clocks": clk}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -609,6 +675,8 @@ def main():
                     help="--decode: key splits per (sequence, K/V head); 0 = automatic")
     ap.add_argument("--layout", action="store_true",
                     help="time the packed-layout helpers (unpad, pad) instead of the forward")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (dQ, dK, dV) instead of the forward")
     ap.add_argument("--sequences", type=int, default=0,
                     help="use only the first N sequences (small case for profiling)")
     args = ap.parse_args()
@@ -621,6 +689,9 @@ def main():
         return
     if args.decode:
         run_decode(args, world, rank, local)
+        return
+    if args.backward:
+        run_backward(args, world, rank, local)
         return
     run_gpu(args, world, rank, local)
 

@@ -29,6 +29,8 @@
 // kernel with atomic dQ accumulation would; in exchange nothing is reduced
 // across CTAs and the results do not depend on scheduling.
 #pragma once
+#include <type_traits>
+
 #include "attn_sm100.cuh"
 
 namespace va {
@@ -68,8 +70,9 @@ struct BwdCfg {
   static constexpr int kStageOff = 2 * kTile;             // two stages of two tiles
   static constexpr int kRowOff = kStageOff + 4 * kTile;   // float [2 buf][2][128]
   static constexpr int kBarOff = kRowOff + 2 * 2 * 128 * 4;
-  // fixed_full, st_full[2], st_empty[2], s_full, p_full, o_full, rows_full[2]
-  static constexpr int kNumBars = 10;
+  // fixed_full, st_full[2], st_empty[2], s_full, p_full, o_full, rows_full[2],
+  // dp_full, ds_full
+  static constexpr int kNumBars = 12;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem slot, abort flag
   static constexpr int kUsed = kMiscOff + 16 + 1024;       // + alignment slack
   // At least 120 KB so that one CTA (holding all 512 tensor-memory columns)
@@ -95,6 +98,8 @@ struct BwdSmem {
   __device__ uint64_t* p_full() const { return bars() + 6; }
   __device__ uint64_t* o_full() const { return bars() + 7; }
   __device__ uint64_t* rows_full(int b) const { return bars() + 8 + b; }
+  __device__ uint64_t* dp_full() const { return bars() + 10; }
+  __device__ uint64_t* ds_full() const { return bars() + 11; }
   __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + BwdCfg<D>::kMiscOff); }
   __device__ int* abort_flag() const { return reinterpret_cast<int*>(base + BwdCfg<D>::kMiscOff + 4); }
 };
@@ -146,6 +151,8 @@ __device__ __forceinline__ uint32_t bwd_setup(BwdSmem<D>& sm, uint8_t* smem_raw)
     ptx::mbar_init(sm.o_full(), 1);
     ptx::mbar_init(sm.rows_full(0), 128);
     ptx::mbar_init(sm.rows_full(1), 128);
+    ptx::mbar_init(sm.dp_full(), 1);
+    ptx::mbar_init(sm.ds_full(), 128);
     *sm.abort_flag() = 0;
     ptx::fence_mbar_init();
   }
@@ -264,34 +271,61 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int st = 0; st < 2; ++st)
       if (uses[st] > 0) drain_bar(sm.st_full(st), (uses[st] - 1) & 1);
   } else if (warp == kBwdMmaWarp) {
+    // Order per tile t: S^T(t), dP^T(t) | P(t) ready: dV(t), S^T(t+1) |
+    // dS(t) ready: dK(t), dP^T(t+1). The compute warps turn S into P while
+    // dP^T(t) runs and dP into dS while dV(t) and S^T(t+1) run. A product
+    // that overwrites columns an earlier product reads is issued after it
+    // (the tensor pipe runs in order).
     const uint64_t kd = desc_kmajor_sw128(ptx::smem_u32(sm.fixed(0)));
     const uint64_t vd = desc_kmajor_sw128(ptx::smem_u32(sm.fixed(1)));
     bool ok = __all_sync(FULL, wait_bar(sm.fixed_full(), 0, ctl));
-    for (int t = 0; t < n_tiles && ok; ++t) {
-      const int st = t & 1;
-      ok = __all_sync(FULL, wait_bar(sm.st_full(st), (t >> 1) & 1, ctl));
-      if (!ok) break;
+    auto stage_addr = [&](int t, int i) { return ptx::smem_u32(sm.stage(t & 1, i)); };
+    auto issue_sT = [&](int t) {  // S^T(t) = K Q(t)^T
+      ok = __all_sync(FULL, wait_bar(sm.st_full(t & 1), (t >> 1) & 1, ctl));
+      if (!ok) return;
       ptx::tc_fence_after();
-      const uint32_t qa = ptx::smem_u32(sm.stage(st, 0)), da = ptx::smem_u32(sm.stage(st, 1));
       if (ptx::elect_one()) {
-        issue_s<D>(tmem + 0, kd, desc_kmajor_sw128(qa));     // S^T  = K Q^T
-        issue_s<D>(tmem + 128, vd, desc_kmajor_sw128(da));   // dP^T = V dO^T
+        issue_s<D>(tmem + 0, kd, desc_kmajor_sw128(stage_addr(t, 0)));
         ptx::tc_commit(sm.s_full());
       }
       __syncwarp();
+    };
+    auto issue_dpT = [&](int t) {  // dP^T(t) = V dO(t)^T
+      if (ptx::elect_one()) {
+        issue_s<D>(tmem + 128, vd, desc_kmajor_sw128(stage_addr(t, 1)));
+        ptx::tc_commit(sm.dp_full());
+      }
+      __syncwarp();
+    };
+    if (n_tiles > 0 && ok) {
+      issue_sT(0);
+      if (ok) issue_dpT(0);
+    }
+    for (int t = 0; t < n_tiles && ok; ++t) {
       ok = __all_sync(FULL, wait_bar(sm.p_full(), t & 1, ctl));
       if (!ok) break;
       ptx::tc_fence_after();
-      if (ptx::elect_one()) {
-        const uint64_t dmn = desc_mnmajor_sw128(da, BwdCfg<D>::kChunk);
-        const uint64_t qmn = desc_mnmajor_sw128(qa, BwdCfg<D>::kChunk);
-        issue_pv_half<D>(tmem + 256, tmem + 0, dmn, 0, t > 0);       // dV += P^T dO
+      if (ptx::elect_one()) {  // dV += P^T dO
+        const uint64_t dmn = desc_mnmajor_sw128(stage_addr(t, 1), BwdCfg<D>::kChunk);
+        issue_pv_half<D>(tmem + 256, tmem + 0, dmn, 0, t > 0);
         issue_pv_half<D>(tmem + 256, tmem + 0, dmn, 1, true);
-        issue_pv_half<D>(tmem + 256 + D, tmem + 128, qmn, 0, t > 0); // dK += dS^T Q
-        issue_pv_half<D>(tmem + 256 + D, tmem + 128, qmn, 1, true);
-        ptx::tc_commit(sm.st_empty(st));
       }
       __syncwarp();
+      if (t + 1 < n_tiles) {
+        issue_sT(t + 1);
+        if (!ok) break;
+      }
+      ok = __all_sync(FULL, wait_bar(sm.ds_full(), t & 1, ctl));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      if (ptx::elect_one()) {  // dK += dS^T Q
+        const uint64_t qmn = desc_mnmajor_sw128(stage_addr(t, 0), BwdCfg<D>::kChunk);
+        issue_pv_half<D>(tmem + 256 + D, tmem + 128, qmn, 0, t > 0);
+        issue_pv_half<D>(tmem + 256 + D, tmem + 128, qmn, 1, true);
+        ptx::tc_commit(sm.st_empty(t & 1));
+      }
+      __syncwarp();
+      if (t + 1 < n_tiles) issue_dpT(t + 1);
     }
     if (ptx::elect_one()) ptx::tc_commit(sm.o_full());
     __syncwarp();
@@ -303,7 +337,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t t_s = tmem + lane_base, t_dp = tmem + lane_base + 128;
     const int kc = kb * BN + c;
     const bool key_ok = kc < Lk;
-    const float kL2 = kLog2e;
     float dbk = 0.f, bkey = 0.f;
     bool ok = true;
     for (int t = 0; t < n_tiles && ok; ++t) {
@@ -318,7 +351,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int b = t & 1;
         const int rl = qb * BM + c;
         const long long gi = (long long)h * p.total_q + q0 + rl;
-        sm.rows(b, 0)[c] = rl < Lq ? p.lse[gi] * kL2 : 0.f;
+        sm.rows(b, 0)[c] = rl < Lq ? p.lse[gi] * kLog2e : 0.f;
         sm.rows(b, 1)[c] = rl < Lq ? p.delta[gi] : 0.f;
         // Buffer b is written again at tile t + 2, after every thread has
         // arrived for tile t + 1, i.e. finished reading it for tile t.
@@ -328,55 +361,98 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       const float* lse2 = sm.rows(t & 1, 0);
       const float* dl = sm.rows(t & 1, 1);
-      ok = __all_sync(FULL, wait_bar(sm.s_full(), t & 1, ctl));
-      if (!ok) break;
-      ptx::tc_fence_after();
+      // every row of the tile sees this key (no mask test per element)
+      const bool full = key_ok && qb * BM + BM <= Lq && (!p.causal || kc <= qb * BM + off);
       const float* grow = nullptr;
       if constexpr (kBiasPair)
         grow = p.bias_pair + (long long)seq * p.sb + (long long)(h / p.bias_head_div) * p.sh +
                (long long)kc * p.sc;
-      float* dgrow = p.dbias_pair == nullptr
-                         ? nullptr
-                         : p.dbias_pair + (long long)seq * p.dsb + (long long)h * p.dsh + kc;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t s[32], dp[32];
-        ptx::tmem_ld32(t_s + cc * 32, s);
-        ptx::tmem_ld32(t_dp + cc * 32, dp);
-        ptx::tmem_wait_ld();
-        uint32_t pk[16], dk16[16];
+      auto visible = [&](int r) {
+        const int ql = qb * BM + r;
+        return full || (key_ok && ql < Lq && (!p.causal || kc <= ql + off));
+      };
+      // pass 1: S^T -> P^T, bf16 (to tensor memory for dV, and kept packed
+      // in registers for dS: 64 registers instead of 128)
+      ok = __all_sync(FULL, wait_bar(sm.s_full(), t & 1, ctl));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      uint32_t pk[BM / 2];
+      // Tiles where every row sees the key skip the per-element mask (the
+      // masked variant is a separate copy of the loop so that its extra
+      // registers do not weigh on the common one).
+      auto pass1 = [&](auto masked) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pv[2], dsv[2];
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t sv[32];
+          ptx::tmem_ld32(t_s + cc * 32, sv);
+          ptx::tmem_wait_ld();
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int r = cc * 32 + e + u;
-            const int ql = qb * BM + r;
-            const bool in = key_ok && ql < Lq;
-            const bool vis = in && (!p.causal || kc <= ql + off);
-            float x = __uint_as_float(s[e + u]) * p.scale;
-            if constexpr (kBiasKey) x += bkey;
-            if constexpr (kBiasPair) {
-              if (vis) x += __ldg(grow + (long long)ql * p.sr);
+          for (int e = 0; e < 32; e += 2) {
+            float pv[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int r = cc * 32 + e + u;
+              float x = __uint_as_float(sv[e + u]) * p.scale;
+              if constexpr (kBiasKey) x += bkey;
+              const bool vis = decltype(masked)::value ? visible(r) : true;
+              if constexpr (kBiasPair) {
+                if (vis) x += __ldg(grow + (long long)(qb * BM + r) * p.sr);
+              }
+              pv[u] = vis ? ptx::ex2(fmaf(x, kLog2e, -lse2[r])) : 0.f;
             }
-            const float pr = vis ? ptx::ex2(fmaf(x, kL2, -lse2[r])) : 0.f;
-            const float ds = pr * (__uint_as_float(dp[e + u]) - dl[r]);
-            dbk += ds;
-            if (dgrow != nullptr && in) dgrow[(long long)ql * p.dsr] = ds;
-            pv[u] = pr;
-            dsv[u] = ds;
+            pk[(cc * 32 + e) / 2] = ptx::pack_bf16x2(pv[0], pv[1]);
           }
-          pk[e / 2] = ptx::pack_bf16x2(pv[0], pv[1]);
-          dk16[e / 2] = ptx::pack_bf16x2(dsv[0], dsv[1]);
+          // P^T(cc) covers columns [16cc, 16cc + 16), already read
+          ptx::tmem_st16(t_s + cc * 16, &pk[cc * 16]);
         }
-        // P^T over S^T and dS^T over dP^T: chunk cc only covers columns
-        // [16cc, 16cc + 16), which were read in this or an earlier chunk.
-        ptx::tmem_st16(t_s + cc * 16, pk);
-        ptx::tmem_st16(t_dp + cc * 16, dk16);
-      }
+      };
+      // (warp-uniform choice: the loop holds warp-collective tensor-memory
+      // loads and stores)
+      if (__all_sync(FULL, full)) pass1(std::false_type{});
+      else pass1(std::true_type{});
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       ptx::mbar_arrive(sm.p_full());
+      // pass 2: dP^T -> dS^T
+      ok = __all_sync(FULL, wait_bar(sm.dp_full(), t & 1, ctl));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      float* dgrow = p.dbias_pair == nullptr
+                         ? nullptr
+                         : p.dbias_pair + (long long)seq * p.dsb + (long long)h * p.dsh + kc;
+      auto pass2 = [&](auto store_grid) {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t dp[32];
+          ptx::tmem_ld32(t_dp + cc * 32, dp);
+          ptx::tmem_wait_ld();
+          uint32_t dk16[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const uint32_t w = pk[(cc * 32 + e) / 2];
+            const float pv[2] = {__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)};
+            float dsv[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int r = cc * 32 + e + u;
+              const float ds = pv[u] * (__uint_as_float(dp[e + u]) - dl[r]);
+              dbk += ds;
+              if constexpr (decltype(store_grid)::value) {
+                const int ql = qb * BM + r;
+                if (key_ok && ql < Lq) dgrow[(long long)ql * p.dsr] = ds;
+              }
+              dsv[u] = ds;
+            }
+            dk16[e / 2] = ptx::pack_bf16x2(dsv[0], dsv[1]);
+          }
+          ptx::tmem_st16(t_dp + cc * 16, dk16);
+        }
+      };
+      if (dgrow != nullptr) pass2(std::true_type{});
+      else pass2(std::false_type{});
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(sm.ds_full());
       if (p.dbias_key != nullptr && key_ok && t % per_head == per_head - 1)
         p.dbias_key[(long long)(k0 + kc) * p.n_heads + h] = dbk;
     }
@@ -446,31 +522,52 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int st = 0; st < 2; ++st)
       if (uses[st] > 0) drain_bar(sm.st_full(st), (uses[st] - 1) & 1);
   } else if (warp == kBwdMmaWarp) {
+    // Order per key tile j: S(j), dP(j) | S(j) read: S(j+1) | dS(j) ready:
+    // dQ(j), dP(j+1). The compute warps turn S into P while dP(j) runs and
+    // dP into dS while S(j+1) runs.
     const uint64_t qd = desc_kmajor_sw128(ptx::smem_u32(sm.fixed(0)));
     const uint64_t dod = desc_kmajor_sw128(ptx::smem_u32(sm.fixed(1)));
     bool ok = n_k == 0 || __all_sync(FULL, wait_bar(sm.fixed_full(), 0, ctl));
-    for (int j = 0; j < n_k && ok; ++j) {
-      const int st = j & 1;
-      ok = __all_sync(FULL, wait_bar(sm.st_full(st), (j >> 1) & 1, ctl));
-      if (!ok) break;
+    auto stage_addr = [&](int j, int i) { return ptx::smem_u32(sm.stage(j & 1, i)); };
+    auto issue_s_j = [&](int j) {  // S(j) = Q K(j)^T
+      ok = __all_sync(FULL, wait_bar(sm.st_full(j & 1), (j >> 1) & 1, ctl));
+      if (!ok) return;
       ptx::tc_fence_after();
-      const uint32_t ka = ptx::smem_u32(sm.stage(st, 0)), va_ = ptx::smem_u32(sm.stage(st, 1));
       if (ptx::elect_one()) {
-        issue_s<D>(tmem + 0, qd, desc_kmajor_sw128(ka));      // S  = Q K^T
-        issue_s<D>(tmem + 128, dod, desc_kmajor_sw128(va_));  // dP = dO V^T
+        issue_s<D>(tmem + 0, qd, desc_kmajor_sw128(stage_addr(j, 0)));
         ptx::tc_commit(sm.s_full());
       }
       __syncwarp();
-      ok = __all_sync(FULL, wait_bar(sm.p_full(), j & 1, ctl));
-      if (!ok) break;
-      ptx::tc_fence_after();
+    };
+    auto issue_dp_j = [&](int j) {  // dP(j) = dO V(j)^T
       if (ptx::elect_one()) {
-        const uint64_t kmn = desc_mnmajor_sw128(ka, BwdCfg<D>::kChunk);
-        issue_pv_half<D>(tmem + 256, tmem + 128, kmn, 0, j > 0);  // dQ += dS K
-        issue_pv_half<D>(tmem + 256, tmem + 128, kmn, 1, true);
-        ptx::tc_commit(sm.st_empty(st));
+        issue_s<D>(tmem + 128, dod, desc_kmajor_sw128(stage_addr(j, 1)));
+        ptx::tc_commit(sm.dp_full());
       }
       __syncwarp();
+    };
+    if (n_k > 0 && ok) {
+      issue_s_j(0);
+      if (ok) issue_dp_j(0);
+    }
+    for (int j = 0; j < n_k && ok; ++j) {
+      ok = __all_sync(FULL, wait_bar(sm.p_full(), j & 1, ctl));  // S(j) has been read
+      if (!ok) break;
+      if (j + 1 < n_k) {
+        issue_s_j(j + 1);
+        if (!ok) break;
+      }
+      ok = __all_sync(FULL, wait_bar(sm.ds_full(), j & 1, ctl));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      if (ptx::elect_one()) {  // dQ += dS K
+        const uint64_t kmn = desc_mnmajor_sw128(stage_addr(j, 0), BwdCfg<D>::kChunk);
+        issue_pv_half<D>(tmem + 256, tmem + 128, kmn, 0, j > 0);
+        issue_pv_half<D>(tmem + 256, tmem + 128, kmn, 1, true);
+        ptx::tc_commit(sm.st_empty(j & 1));
+      }
+      __syncwarp();
+      if (j + 1 < n_k) issue_dp_j(j + 1);
     }
     if (ptx::elect_one()) ptx::tc_commit(sm.o_full());
     __syncwarp();
@@ -491,40 +588,51 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
              (long long)ql * p.sr;
     bool ok = true;
     for (int j = 0; j < n_k && ok; ++j) {
+      // every key of the tile is visible to this row (no mask test per element)
+      const bool full = row_ok && j * BN + BN <= Lk && (!p.causal || j * BN + BN - 1 <= ql + off);
       ok = __all_sync(FULL, wait_bar(sm.s_full(), j & 1, ctl));
       if (!ok) break;
       ptx::tc_fence_after();
-#pragma unroll 1
+      float pr[BN];
+#pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        uint32_t s[32], dp[32];
-        ptx::tmem_ld32(t_s + cc * 32, s);
+        uint32_t sv[32];
+        ptx::tmem_ld32(t_s + cc * 32, sv);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int kc = j * BN + cc * 32 + e;
+          const bool vis = full || (row_ok && kc < Lk && (!p.causal || kc <= ql + off));
+          float x = __uint_as_float(sv[e]) * p.scale;
+          if constexpr (kBiasKey) {
+            if (vis) x += __ldg(p.bias_key + (long long)(k0 + kc) * p.n_heads + h);
+          }
+          if constexpr (kBiasPair) {
+            if (vis) x += __ldg(grow + (long long)kc * p.sc);
+          }
+          pr[cc * 32 + e] = vis ? ptx::ex2(fmaf(x, kLog2e, -lse2)) : 0.f;
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(sm.p_full());  // S(j) read: the next S may overwrite it
+      ok = __all_sync(FULL, wait_bar(sm.dp_full(), j & 1, ctl));
+      if (!ok) break;
+      ptx::tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t dp[32];
         ptx::tmem_ld32(t_dp + cc * 32, dp);
         ptx::tmem_wait_ld();
         uint32_t dk16[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float dsv[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int kc = j * BN + cc * 32 + e + u;
-            const bool vis = row_ok && kc < Lk && (!p.causal || kc <= ql + off);
-            float x = __uint_as_float(s[e + u]) * p.scale;
-            if constexpr (kBiasKey) {
-              if (vis) x += __ldg(p.bias_key + (long long)(k0 + kc) * p.n_heads + h);
-            }
-            if constexpr (kBiasPair) {
-              if (vis) x += __ldg(grow + (long long)kc * p.sc);
-            }
-            const float pr = vis ? ptx::ex2(fmaf(x, kLog2e, -lse2)) : 0.f;
-            dsv[u] = pr * (__uint_as_float(dp[e + u]) - dl);
-          }
-          dk16[e / 2] = ptx::pack_bf16x2(dsv[0], dsv[1]);
-        }
+        for (int e = 0; e < 32; e += 2)
+          dk16[e / 2] = ptx::pack_bf16x2(pr[cc * 32 + e] * (__uint_as_float(dp[e]) - dl),
+                                         pr[cc * 32 + e + 1] * (__uint_as_float(dp[e + 1]) - dl));
         ptx::tmem_st16(t_dp + cc * 16, dk16);
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(sm.p_full());
+      ptx::mbar_arrive(sm.ds_full());
     }
     const bool have = n_k > 0;
     if (have) {
