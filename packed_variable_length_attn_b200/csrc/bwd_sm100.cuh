@@ -58,9 +58,13 @@ struct BwdParams {
   int* error;
 };
 
-constexpr int kBwdThreads = 192;  // compute warps 0-3, MMA warp 4, load warp 5
-constexpr int kBwdMmaWarp = 4;
-constexpr int kBwdLoadWarp = 5;
+// Compute warps 0-7: warp w reads tensor-memory lanes 32(w % 4) .. +31 and
+// the half w / 4 of each 128-column tile (two warps per SM sub-partition).
+// MMA warp 8, load warp 9.
+constexpr int kBwdThreads = 320;
+constexpr int kBwdCompute = 256;
+constexpr int kBwdMmaWarp = 8;
+constexpr int kBwdLoadWarp = 9;
 
 template <int D>
 struct BwdCfg {
@@ -147,12 +151,12 @@ __device__ __forceinline__ uint32_t bwd_setup(BwdSmem<D>& sm, uint8_t* smem_raw)
       ptx::mbar_init(sm.st_empty(st), 1);
     }
     ptx::mbar_init(sm.s_full(), 1);
-    ptx::mbar_init(sm.p_full(), 128);
+    ptx::mbar_init(sm.p_full(), kBwdCompute);
     ptx::mbar_init(sm.o_full(), 1);
-    ptx::mbar_init(sm.rows_full(0), 128);
-    ptx::mbar_init(sm.rows_full(1), 128);
+    ptx::mbar_init(sm.rows_full(0), kBwdCompute);
+    ptx::mbar_init(sm.rows_full(1), kBwdCompute);
     ptx::mbar_init(sm.dp_full(), 1);
-    ptx::mbar_init(sm.ds_full(), 128);
+    ptx::mbar_init(sm.ds_full(), kBwdCompute);
     *sm.abort_flag() = 0;
     ptx::fence_mbar_init();
   }
@@ -187,11 +191,11 @@ __device__ __forceinline__ void bwd_load_tile(uint8_t* dst, const CUtensorMap* t
 
 // Accumulator rows of tensor memory (D fp32 columns at `t`) -> bf16 row of
 // `dst` times `mul`, or zeros when `have` is false.
-template <int D>
+template <int C0, int C1>
 __device__ __forceinline__ void bwd_store_row(uint32_t t, bool have, float mul, __nv_bfloat16* dst,
                                               bool ok) {
 #pragma unroll
-  for (int c = 0; c < D / 32; ++c) {
+  for (int c = C0; c < C1; ++c) {
     uint32_t v[32];
     if (have) {
       ptx::tmem_ld32(t + c * 32, v);
@@ -308,7 +312,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (ptx::elect_one()) {  // dV += P^T dO
         const uint64_t dmn = desc_mnmajor_sw128(stage_addr(t, 1), BwdCfg<D>::kChunk);
         issue_pv_half<D>(tmem + 256, tmem + 0, dmn, 0, t > 0);
-        issue_pv_half<D>(tmem + 256, tmem + 0, dmn, 1, true);
+        issue_pv_half<D>(tmem + 256, tmem + 32, dmn, 1, true);  // rows 64.. at cols [64, 96)
       }
       __syncwarp();
       if (t + 1 < n_tiles) {
@@ -321,7 +325,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (ptx::elect_one()) {  // dK += dS^T Q
         const uint64_t qmn = desc_mnmajor_sw128(stage_addr(t, 0), BwdCfg<D>::kChunk);
         issue_pv_half<D>(tmem + 256 + D, tmem + 128, qmn, 0, t > 0);
-        issue_pv_half<D>(tmem + 256 + D, tmem + 128, qmn, 1, true);
+        issue_pv_half<D>(tmem + 256 + D, tmem + 160, qmn, 1, true);
         ptx::tc_commit(sm.st_empty(t & 1));
       }
       __syncwarp();
@@ -331,10 +335,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
     drain_bar(sm.o_full(), 0);
   } else {
-    // compute warps: thread c owns key kb*BN + c (tensor-memory lane c)
-    const int c = threadIdx.x;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t t_s = tmem + lane_base, t_dp = tmem + lane_base + 128;
+    // compute warps: thread (c, hh) owns key kb*BN + c (tensor-memory lane c)
+    // and the query rows [64hh, 64hh + 64) of every tile
+    const int lane = threadIdx.x & 31;
+    const int c = (warp & 3) * 32 + lane, hh = warp >> 2, r0 = hh * 64;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem + lane_base + r0, t_dp = tmem + lane_base + 128 + r0;
     const int kc = kb * BN + c;
     const bool key_ok = kc < Lk;
     float dbk = 0.f, bkey = 0.f;
@@ -346,13 +352,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         dbk = 0.f;
         if constexpr (kBiasKey) bkey = key_ok ? p.bias_key[(long long)(k0 + kc) * p.n_heads + h] : 0.f;
       }
-      // this tile's row constants: LSE * log2(e) and delta
+      // this tile's row constants: LSE * log2(e) and delta (written by the
+      // first 128 threads, read by all)
       {
         const int b = t & 1;
-        const int rl = qb * BM + c;
-        const long long gi = (long long)h * p.total_q + q0 + rl;
-        sm.rows(b, 0)[c] = rl < Lq ? p.lse[gi] * kLog2e : 0.f;
-        sm.rows(b, 1)[c] = rl < Lq ? p.delta[gi] : 0.f;
+        if (hh == 0) {
+          const int rl = qb * BM + c;
+          const long long gi = (long long)h * p.total_q + q0 + rl;
+          sm.rows(b, 0)[c] = rl < Lq ? p.lse[gi] * kLog2e : 0.f;
+          sm.rows(b, 1)[c] = rl < Lq ? p.delta[gi] : 0.f;
+        }
         // Buffer b is written again at tile t + 2, after every thread has
         // arrived for tile t + 1, i.e. finished reading it for tile t.
         ptx::mbar_arrive(sm.rows_full(b));
@@ -361,28 +370,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       const float* lse2 = sm.rows(t & 1, 0);
       const float* dl = sm.rows(t & 1, 1);
-      // every row of the tile sees this key (no mask test per element)
-      const bool full = key_ok && qb * BM + BM <= Lq && (!p.causal || kc <= qb * BM + off);
+      // every row of this thread's half sees the key (no per-element mask)
+      const bool full = key_ok && qb * BM + r0 + 64 <= Lq && (!p.causal || kc <= qb * BM + r0 + off);
       const float* grow = nullptr;
       if constexpr (kBiasPair)
         grow = p.bias_pair + (long long)seq * p.sb + (long long)(h / p.bias_head_div) * p.sh +
                (long long)kc * p.sc;
       auto visible = [&](int r) {
         const int ql = qb * BM + r;
-        return full || (key_ok && ql < Lq && (!p.causal || kc <= ql + off));
+        return key_ok && ql < Lq && (!p.causal || kc <= ql + off);
       };
-      // pass 1: S^T -> P^T, bf16 (to tensor memory for dV, and kept packed
-      // in registers for dS: 64 registers instead of 128)
+      // pass 1: S^T -> P^T, bf16 (to tensor memory for dV, over this half's
+      // own S^T columns, and kept packed in registers for dS)
       ok = __all_sync(FULL, wait_bar(sm.s_full(), t & 1, ctl));
       if (!ok) break;
       ptx::tc_fence_after();
-      uint32_t pk[BM / 2];
-      // Tiles where every row sees the key skip the per-element mask (the
-      // masked variant is a separate copy of the loop so that its extra
-      // registers do not weigh on the common one).
+      uint32_t pk[32];
       auto pass1 = [&](auto masked) {
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < 2; ++cc) {
           uint32_t sv[32];
           ptx::tmem_ld32(t_s + cc * 32, sv);
           ptx::tmem_wait_ld();
@@ -391,7 +397,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             float pv[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
-              const int r = cc * 32 + e + u;
+              const int r = r0 + cc * 32 + e + u;
               float x = __uint_as_float(sv[e + u]) * p.scale;
               if constexpr (kBiasKey) x += bkey;
               const bool vis = decltype(masked)::value ? visible(r) : true;
@@ -402,7 +408,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             pk[(cc * 32 + e) / 2] = ptx::pack_bf16x2(pv[0], pv[1]);
           }
-          // P^T(cc) covers columns [16cc, 16cc + 16), already read
+          // columns [r0 + 16cc, +16): this half's, already read
           ptx::tmem_st16(t_s + cc * 16, &pk[cc * 16]);
         }
       };
@@ -422,7 +428,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                          : p.dbias_pair + (long long)seq * p.dsb + (long long)h * p.dsh + kc;
       auto pass2 = [&](auto store_grid) {
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < 2; ++cc) {
           uint32_t dp[32];
           ptx::tmem_ld32(t_dp + cc * 32, dp);
           ptx::tmem_wait_ld();
@@ -434,7 +440,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             float dsv[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
-              const int r = cc * 32 + e + u;
+              const int r = r0 + cc * 32 + e + u;
               const float ds = pv[u] * (__uint_as_float(dp[e + u]) - dl[r]);
               dbk += ds;
               if constexpr (decltype(store_grid)::value) {
@@ -453,22 +459,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       ptx::mbar_arrive(sm.ds_full());
+      // two halves add into the zeroed output: 0 + a + b in either order is
+      // the same fp32 value, so the result stays deterministic
       if (p.dbias_key != nullptr && key_ok && t % per_head == per_head - 1)
-        p.dbias_key[(long long)(k0 + kc) * p.n_heads + h] = dbk;
+        atomicAdd(p.dbias_key + (long long)(k0 + kc) * p.n_heads + h, dbk);
     }
-    if (ok && p.dbias_key != nullptr && key_ok && per_head == 0)
-      for (int g = 0; g < G; ++g) p.dbias_key[(long long)(k0 + kc) * p.n_heads + kvh * G + g] = 0.f;
     const bool have = n_tiles > 0;
     if (have) {
       ok = ok && __all_sync(FULL, wait_bar(sm.o_full(), 0, ctl));
       ptx::tc_fence_after();
     }
-    if (ok) {
+    if (ok) {  // half 0 writes dV, half 1 dK
       const long long o = ((long long)(k0 + kc) * p.n_kv_heads + kvh) * D;
-      bwd_store_row<D>(tmem + lane_base + 256, have, 1.f,
-                       reinterpret_cast<__nv_bfloat16*>(p.dv) + o, key_ok);
-      bwd_store_row<D>(tmem + lane_base + 256 + D, have, p.scale,
-                       reinterpret_cast<__nv_bfloat16*>(p.dk) + o, key_ok);
+      if (hh == 0)
+        bwd_store_row<0, D / 32>(tmem + lane_base + 256, have, 1.f,
+                                 reinterpret_cast<__nv_bfloat16*>(p.dv) + o, key_ok);
+      else
+        bwd_store_row<0, D / 32>(tmem + lane_base + 256 + D, have, p.scale,
+                                 reinterpret_cast<__nv_bfloat16*>(p.dk) + o, key_ok);
     }
   }
   bwd_teardown<D>(sm, tmem);
@@ -563,7 +571,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (ptx::elect_one()) {  // dQ += dS K
         const uint64_t kmn = desc_mnmajor_sw128(stage_addr(j, 0), BwdCfg<D>::kChunk);
         issue_pv_half<D>(tmem + 256, tmem + 128, kmn, 0, j > 0);
-        issue_pv_half<D>(tmem + 256, tmem + 128, kmn, 1, true);
+        issue_pv_half<D>(tmem + 256, tmem + 160, kmn, 1, true);  // keys 64.. at cols [192, 224)
         ptx::tc_commit(sm.st_empty(j & 1));
       }
       __syncwarp();
@@ -573,10 +581,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
     drain_bar(sm.o_full(), 0);
   } else {
-    // compute warps: thread r owns query row qb*BM + r
-    const int r = threadIdx.x;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t t_s = tmem + lane_base, t_dp = tmem + lane_base + 128;
+    // compute warps: thread (r, hh) owns query row qb*BM + r and the keys
+    // [64hh, 64hh + 64) of every tile
+    const int lane = threadIdx.x & 31;
+    const int r = (warp & 3) * 32 + lane, hh = warp >> 2, c0 = hh * 64;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem + lane_base + c0, t_dp = tmem + lane_base + 128 + c0;
     const int ql = qb * BM + r;
     const bool row_ok = ql < Lq;
     const long long gi = (long long)h * p.total_q + q0 + ql;
@@ -588,20 +598,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
              (long long)ql * p.sr;
     bool ok = true;
     for (int j = 0; j < n_k && ok; ++j) {
-      // every key of the tile is visible to this row (no mask test per element)
-      const bool full = row_ok && j * BN + BN <= Lk && (!p.causal || j * BN + BN - 1 <= ql + off);
+      const int kt = j * BN + c0;  // this half's first key
+      // every key of this half is visible to the row (no per-element mask)
+      const bool full = row_ok && kt + 64 <= Lk && (!p.causal || kt + 63 <= ql + off);
       ok = __all_sync(FULL, wait_bar(sm.s_full(), j & 1, ctl));
       if (!ok) break;
       ptx::tc_fence_after();
-      float pr[BN];
+      float pr[64];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t sv[32];
         ptx::tmem_ld32(t_s + cc * 32, sv);
         ptx::tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const int kc = j * BN + cc * 32 + e;
+          const int kc = kt + cc * 32 + e;
           const bool vis = full || (row_ok && kc < Lk && (!p.causal || kc <= ql + off));
           float x = __uint_as_float(sv[e]) * p.scale;
           if constexpr (kBiasKey) {
@@ -619,7 +630,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ok) break;
       ptx::tc_fence_after();
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t dp[32];
         ptx::tmem_ld32(t_dp + cc * 32, dp);
         ptx::tmem_wait_ld();
@@ -628,6 +639,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int e = 0; e < 32; e += 2)
           dk16[e / 2] = ptx::pack_bf16x2(pr[cc * 32 + e] * (__uint_as_float(dp[e]) - dl),
                                          pr[cc * 32 + e + 1] * (__uint_as_float(dp[e + 1]) - dl));
+        // columns [128 + c0 + 16cc, +16): this half's, already read
         ptx::tmem_st16(t_dp + cc * 16, dk16);
       }
       ptx::tmem_wait_st();
@@ -639,10 +651,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = ok && __all_sync(FULL, wait_bar(sm.o_full(), 0, ctl));
       ptx::tc_fence_after();
     }
-    if (ok)
-      bwd_store_row<D>(tmem + lane_base + 256, have, p.scale,
-                       reinterpret_cast<__nv_bfloat16*>(p.dq) + ((long long)(q0 + ql) * p.n_heads + h) * D,
-                       row_ok);
+    if (ok) {  // half hh writes columns [hh * D/2, (hh + 1) * D/2) of the row
+      __nv_bfloat16* dst =
+          reinterpret_cast<__nv_bfloat16*>(p.dq) + ((long long)(q0 + ql) * p.n_heads + h) * D;
+      if (hh == 0)
+        bwd_store_row<0, D / 64>(tmem + lane_base + 256, have, p.scale, dst, row_ok);
+      else
+        bwd_store_row<D / 64, D / 32>(tmem + lane_base + 256, have, p.scale, dst, row_ok);
+    }
   }
   bwd_teardown<D>(sm, tmem);
 }

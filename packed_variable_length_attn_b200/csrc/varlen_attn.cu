@@ -919,6 +919,10 @@ int varlen_attn_bwd(const void* q, const void* k, const void* v, const void* out
       !make_tmap(&tv, v, head_dim, n_kv_heads, total_k, BN))
     return VARLEN_ATTN_ERR_CUDA;
 
+  if (dbias_per_key) {  // the dK/dV kernel adds two half sums per (key, head)
+    cudaError_t e = cudaMemsetAsync(dbias_per_key, 0, (size_t)total_k * n_heads * 4, st);
+    if (e != cudaSuccess) return cuda_fail("cudaMemsetAsync(dbias_per_key)", e);
+  }
   BwdParams bp;
   bp.cu_q = cu_seqlens_q;
   bp.cu_k = cu_seqlens_k;
