@@ -491,7 +491,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                       const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const unsigned FULL = 0xffffffffu;
-  const int qb = blockIdx.x, h = blockIdx.y, seq = blockIdx.z;
+  // Causal rows see more keys the later they are: the last query blocks go
+  // first, so that the longest CTAs do not form the tail of the launch.
+  const int qb = gridDim.x - 1 - blockIdx.x, h = blockIdx.y, seq = blockIdx.z;
   const int q0 = p.cu_q[seq], k0 = p.cu_k[seq];
   const int Lq = p.cu_q[seq + 1] - q0, Lk = p.cu_k[seq + 1] - k0;
   if (*p.valid == 0 || qb * BM >= Lq) return;  // uniform over the CTA, before any barrier
@@ -531,8 +533,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (uses[st] > 0) drain_bar(sm.st_full(st), (uses[st] - 1) & 1);
   } else if (warp == kBwdMmaWarp) {
     // Order per key tile j: S(j), dP(j) | S(j) read: S(j+1) | dS(j) ready:
-    // dQ(j), dP(j+1). The compute warps turn S into P while dP(j) runs and
-    // dP into dS while S(j+1) runs.
+    // dP(j+1), dQ(j). The compute warps turn S into P while dP(j) runs and
+    // dP into dS while S(j+1) runs. dS(j) goes to tensor-memory columns
+    // [384 + 64(j % 2), +64) (free in this kernel), so dP(j+1) need not wait
+    // for dQ(j) to have read it; dS(j+2) is written after dp_full(j+2),
+    // which dQ(j) precedes.
     const uint64_t qd = desc_kmajor_sw128(ptx::smem_u32(sm.fixed(0)));
     const uint64_t dod = desc_kmajor_sw128(ptx::smem_u32(sm.fixed(1)));
     bool ok = n_k == 0 || __all_sync(FULL, wait_bar(sm.fixed_full(), 0, ctl));
@@ -568,14 +573,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(FULL, wait_bar(sm.ds_full(), j & 1, ctl));
       if (!ok) break;
       ptx::tc_fence_after();
+      if (j + 1 < n_k) issue_dp_j(j + 1);
       if (ptx::elect_one()) {  // dQ += dS K
         const uint64_t kmn = desc_mnmajor_sw128(stage_addr(j, 0), BwdCfg<D>::kChunk);
-        issue_pv_half<D>(tmem + 256, tmem + 128, kmn, 0, j > 0);
-        issue_pv_half<D>(tmem + 256, tmem + 160, kmn, 1, true);  // keys 64.. at cols [192, 224)
+        const uint32_t ds_col = tmem + 384 + 64 * (j & 1);
+        issue_pv_half<D>(tmem + 256, ds_col, kmn, 0, j > 0);
+        issue_pv_half<D>(tmem + 256, ds_col, kmn, 1, true);
         ptx::tc_commit(sm.st_empty(j & 1));
       }
       __syncwarp();
-      if (j + 1 < n_k) issue_dp_j(j + 1);
     }
     if (ptx::elect_one()) ptx::tc_commit(sm.o_full());
     __syncwarp();
@@ -605,25 +611,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ok) break;
       ptx::tc_fence_after();
       float pr[64];
+      auto pass1 = [&](auto masked) {
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t sv[32];
-        ptx::tmem_ld32(t_s + cc * 32, sv);
-        ptx::tmem_wait_ld();
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t sv[32];
+          ptx::tmem_ld32(t_s + cc * 32, sv);
+          ptx::tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int kc = kt + cc * 32 + e;
-          const bool vis = full || (row_ok && kc < Lk && (!p.causal || kc <= ql + off));
-          float x = __uint_as_float(sv[e]) * p.scale;
-          if constexpr (kBiasKey) {
-            if (vis) x += __ldg(p.bias_key + (long long)(k0 + kc) * p.n_heads + h);
+          for (int e = 0; e < 32; ++e) {
+            const int kc = kt + cc * 32 + e;
+            const bool vis = decltype(masked)::value
+                                 ? row_ok && kc < Lk && (!p.causal || kc <= ql + off)
+                                 : true;
+            float x = __uint_as_float(sv[e]) * p.scale;
+            if constexpr (kBiasKey) {
+              if (vis) x += __ldg(p.bias_key + (long long)(k0 + kc) * p.n_heads + h);
+            }
+            if constexpr (kBiasPair) {
+              if (vis) x += __ldg(grow + (long long)kc * p.sc);
+            }
+            pr[cc * 32 + e] = vis ? ptx::ex2(fmaf(x, kLog2e, -lse2)) : 0.f;
           }
-          if constexpr (kBiasPair) {
-            if (vis) x += __ldg(grow + (long long)kc * p.sc);
-          }
-          pr[cc * 32 + e] = vis ? ptx::ex2(fmaf(x, kLog2e, -lse2)) : 0.f;
         }
-      }
+      };
+      // (warp-uniform choice: the loop holds warp-collective loads)
+      if (__all_sync(FULL, full)) pass1(std::false_type{});
+      else pass1(std::true_type{});
       ptx::tc_fence_before();
       ptx::mbar_arrive(sm.p_full());  // S(j) read: the next S may overwrite it
       ok = __all_sync(FULL, wait_bar(sm.dp_full(), j & 1, ctl));
@@ -639,8 +652,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int e = 0; e < 32; e += 2)
           dk16[e / 2] = ptx::pack_bf16x2(pr[cc * 32 + e] * (__uint_as_float(dp[e]) - dl),
                                          pr[cc * 32 + e + 1] * (__uint_as_float(dp[e + 1]) - dl));
-        // columns [128 + c0 + 16cc, +16): this half's, already read
-        ptx::tmem_st16(t_dp + cc * 16, dk16);
+        ptx::tmem_st16(tmem + lane_base + 384 + 64 * (j & 1) + hh * 32 + cc * 16, dk16);
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
