@@ -387,11 +387,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ptx::tc_fence_after();
       uint32_t pk[32];
       auto pass1 = [&](auto masked) {
+        uint32_t sv2[2][32];  // both chunks in flight before the first wait
+        ptx::tmem_ld32(t_s, sv2[0]);
+        ptx::tmem_ld32(t_s + 32, sv2[1]);
+        ptx::tmem_wait_ld();
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
-          uint32_t sv[32];
-          ptx::tmem_ld32(t_s + cc * 32, sv);
-          ptx::tmem_wait_ld();
+          uint32_t (&sv)[32] = sv2[cc];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             float pv[2];
@@ -427,11 +429,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                          ? nullptr
                          : p.dbias_pair + (long long)seq * p.dsb + (long long)h * p.dsh + kc;
       auto pass2 = [&](auto store_grid) {
+        uint32_t dp2[2][32];  // both chunks in flight before the first wait
+        ptx::tmem_ld32(t_dp, dp2[0]);
+        ptx::tmem_ld32(t_dp + 32, dp2[1]);
+        ptx::tmem_wait_ld();
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
-          uint32_t dp[32];
-          ptx::tmem_ld32(t_dp + cc * 32, dp);
-          ptx::tmem_wait_ld();
+          uint32_t (&dp)[32] = dp2[cc];
           uint32_t dk16[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
@@ -612,11 +616,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ptx::tc_fence_after();
       float pr[64];
       auto pass1 = [&](auto masked) {
+        uint32_t sv2[2][32];  // both chunks in flight before the first wait
+        ptx::tmem_ld32(t_s, sv2[0]);
+        ptx::tmem_ld32(t_s + 32, sv2[1]);
+        ptx::tmem_wait_ld();
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
-          uint32_t sv[32];
-          ptx::tmem_ld32(t_s + cc * 32, sv);
-          ptx::tmem_wait_ld();
+          uint32_t (&sv)[32] = sv2[cc];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int kc = kt + cc * 32 + e;
@@ -642,11 +648,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(FULL, wait_bar(sm.dp_full(), j & 1, ctl));
       if (!ok) break;
       ptx::tc_fence_after();
+      uint32_t dp2[2][32];  // both chunks in flight before the first wait
+      ptx::tmem_ld32(t_dp, dp2[0]);
+      ptx::tmem_ld32(t_dp + 32, dp2[1]);
+      ptx::tmem_wait_ld();
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        uint32_t dp[32];
-        ptx::tmem_ld32(t_dp + cc * 32, dp);
-        ptx::tmem_wait_ld();
+        uint32_t (&dp)[32] = dp2[cc];
         uint32_t dk16[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2)
