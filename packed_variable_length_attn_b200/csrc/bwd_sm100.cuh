@@ -66,17 +66,31 @@ constexpr int kBwdCompute = 256;
 constexpr int kBwdMmaWarp = 8;
 constexpr int kBwdLoadWarp = 9;
 
+// Stages of the two streamed-operand rings (see BwdCfg): 192 KB of shared
+// memory in all at head_dim 128, 160 KB at 64.
+template <int D>
+constexpr int kBwdRingA = D == 64 ? 4 : 3;
+template <int D>
+constexpr int kBwdRingB = D == 64 ? 4 : 1;
+
 template <int D>
 struct BwdCfg {
   static constexpr int kChunk = 128 * 128;               // 128 rows x 64 bf16 (128 B)
   static constexpr int kTile = (D / 64) * kChunk;         // 128 rows x D bf16
+  // Two streamed operands with rings of their own: A is read by the first
+  // and the last product of a tile (Q in dK/dV: S^T and dK; K in dQ: S and
+  // dQ), so its stage is freed late and it gets the deeper ring; B is read
+  // by products in the middle (dO: dP^T, dV; V: dP) and is freed earlier.
+  static constexpr int kNA = kBwdRingA<D>;
+  static constexpr int kNB = kBwdRingB<D>;
   static constexpr int kFixedOff = 0;                     // two resident tiles
-  static constexpr int kStageOff = 2 * kTile;             // two stages of two tiles
-  static constexpr int kRowOff = kStageOff + 4 * kTile;   // float [2 buf][2][128]
+  static constexpr int kAOff = 2 * kTile;
+  static constexpr int kBOff = kAOff + kNA * kTile;
+  static constexpr int kRowOff = kBOff + kNB * kTile;     // float [2 buf][2][128]
   static constexpr int kBarOff = kRowOff + 2 * 2 * 128 * 4;
-  // fixed_full, st_full[2], st_empty[2], s_full, p_full, o_full, rows_full[2],
-  // dp_full, ds_full
-  static constexpr int kNumBars = 12;
+  // fixed_full, s_full, p_full, o_full, rows_full[2], dp_full, ds_full,
+  // a_full[kNA], a_empty[kNA], b_full[kNB], b_empty[kNB]
+  static constexpr int kNumBars = 8 + 2 * kNA + 2 * kNB;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem slot, abort flag
   static constexpr int kUsed = kMiscOff + 16 + 1024;       // + alignment slack
   // At least 120 KB so that one CTA (holding all 512 tensor-memory columns)
@@ -88,22 +102,25 @@ template <int D>
 struct BwdSmem {
   uint8_t* base;
   __device__ uint8_t* fixed(int i) const { return base + BwdCfg<D>::kFixedOff + i * BwdCfg<D>::kTile; }
-  __device__ uint8_t* stage(int st, int i) const {
-    return base + BwdCfg<D>::kStageOff + (2 * st + i) * BwdCfg<D>::kTile;
-  }
+  __device__ uint8_t* ring_a(int st) const { return base + BwdCfg<D>::kAOff + st * BwdCfg<D>::kTile; }
+  __device__ uint8_t* ring_b(int st) const { return base + BwdCfg<D>::kBOff + st * BwdCfg<D>::kTile; }
   __device__ float* rows(int b, int i) const {
     return reinterpret_cast<float*>(base + BwdCfg<D>::kRowOff) + (2 * b + i) * 128;
   }
   __device__ uint64_t* bars() const { return reinterpret_cast<uint64_t*>(base + BwdCfg<D>::kBarOff); }
   __device__ uint64_t* fixed_full() const { return bars(); }
-  __device__ uint64_t* st_full(int st) const { return bars() + 1 + st; }
-  __device__ uint64_t* st_empty(int st) const { return bars() + 3 + st; }
-  __device__ uint64_t* s_full() const { return bars() + 5; }
-  __device__ uint64_t* p_full() const { return bars() + 6; }
-  __device__ uint64_t* o_full() const { return bars() + 7; }
-  __device__ uint64_t* rows_full(int b) const { return bars() + 8 + b; }
-  __device__ uint64_t* dp_full() const { return bars() + 10; }
-  __device__ uint64_t* ds_full() const { return bars() + 11; }
+  __device__ uint64_t* s_full() const { return bars() + 1; }
+  __device__ uint64_t* p_full() const { return bars() + 2; }
+  __device__ uint64_t* o_full() const { return bars() + 3; }
+  __device__ uint64_t* rows_full(int b) const { return bars() + 4 + b; }
+  __device__ uint64_t* dp_full() const { return bars() + 6; }
+  __device__ uint64_t* ds_full() const { return bars() + 7; }
+  __device__ uint64_t* a_full(int st) const { return bars() + 8 + st; }
+  __device__ uint64_t* a_empty(int st) const { return bars() + 8 + BwdCfg<D>::kNA + st; }
+  __device__ uint64_t* b_full(int st) const { return bars() + 8 + 2 * BwdCfg<D>::kNA + st; }
+  __device__ uint64_t* b_empty(int st) const {
+    return bars() + 8 + 2 * BwdCfg<D>::kNA + BwdCfg<D>::kNB + st;
+  }
   __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + BwdCfg<D>::kMiscOff); }
   __device__ int* abort_flag() const { return reinterpret_cast<int*>(base + BwdCfg<D>::kMiscOff + 4); }
 };
@@ -146,9 +163,13 @@ __device__ __forceinline__ uint32_t bwd_setup(BwdSmem<D>& sm, uint8_t* smem_raw)
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     ptx::mbar_init(sm.fixed_full(), 1);
-    for (int st = 0; st < 2; ++st) {
-      ptx::mbar_init(sm.st_full(st), 1);
-      ptx::mbar_init(sm.st_empty(st), 1);
+    for (int st = 0; st < BwdCfg<D>::kNA; ++st) {
+      ptx::mbar_init(sm.a_full(st), 1);
+      ptx::mbar_init(sm.a_empty(st), 1);
+    }
+    for (int st = 0; st < BwdCfg<D>::kNB; ++st) {
+      ptx::mbar_init(sm.b_full(st), 1);
+      ptx::mbar_init(sm.b_empty(st), 1);
     }
     ptx::mbar_init(sm.s_full(), 1);
     ptx::mbar_init(sm.p_full(), kBwdCompute);
@@ -179,6 +200,12 @@ __device__ __forceinline__ void bwd_teardown(const BwdSmem<D>& sm, uint32_t tmem
     ptx::tmem_dealloc(tmem, 512);
   }
 }
+
+// Position of use u in a ring of N stages: stage and mbarrier parity.
+template <int N>
+__device__ __forceinline__ int ring_stage(int u) { return u % N; }
+template <int N>
+__device__ __forceinline__ uint32_t ring_parity(int u) { return (uint32_t)((u / N) & 1); }
 
 // Loads a 128-row x D tile (D/64 swizzled chunks) at (head, row).
 template <int D>
@@ -219,6 +246,42 @@ __device__ __forceinline__ void bwd_store_row(uint32_t t, bool have, float mul, 
   }
 }
 
+// The load warp's stream: for t = 0 .. n-1, tile t of operand A (ring A)
+// then of operand B (ring B), each once its stage is free; `where(t, head,
+// row)` gives the tensor-map coordinates. Afterwards, waits (bounded,
+// ignoring an abort) for the last copy into every stage it used.
+template <int D, typename Where>
+__device__ __forceinline__ void bwd_stream(const BwdSmem<D>& sm, const CUtensorMap* tm_a,
+                                           const CUtensorMap* tm_b, int n, const Ctl& ctl,
+                                           Where where) {
+  using C = BwdCfg<D>;
+  const unsigned FULL = 0xffffffffu;
+  int na = 0, nb = 0;  // copies issued per ring
+  for (int t = 0; t < n; ++t) {
+    int head, row;
+    where(t, head, row);
+    const int sa = ring_stage<C::kNA>(t), sb = ring_stage<C::kNB>(t);
+    if (!__all_sync(FULL, wait_bar(sm.a_empty(sa), ring_parity<C::kNA>(t) ^ 1, ctl))) break;
+    if (ptx::elect_one()) {
+      ptx::mbar_arrive_expect_tx(sm.a_full(sa), C::kTile);
+      bwd_load_tile<D>(sm.ring_a(sa), tm_a, sm.a_full(sa), head, row);
+    }
+    __syncwarp();
+    ++na;
+    if (!__all_sync(FULL, wait_bar(sm.b_empty(sb), ring_parity<C::kNB>(t) ^ 1, ctl))) break;
+    if (ptx::elect_one()) {
+      ptx::mbar_arrive_expect_tx(sm.b_full(sb), C::kTile);
+      bwd_load_tile<D>(sm.ring_b(sb), tm_b, sm.b_full(sb), head, row);
+    }
+    __syncwarp();
+    ++nb;
+  }
+  for (int st = 0; st < C::kNA && st < na; ++st)
+    drain_bar(sm.a_full(st), ring_parity<C::kNA>(st + ((na - 1 - st) / C::kNA) * C::kNA));
+  for (int st = 0; st < C::kNB && st < nb; ++st)
+    drain_bar(sm.b_full(st), ring_parity<C::kNB>(st + ((nb - 1 - st) / C::kNB) * C::kNB));
+}
+
 // ------------------------------------------------------------------ dK, dV
 template <int D, bool kBiasKey, bool kBiasPair>
 __global__ void __launch_bounds__(kBwdThreads, 1)
@@ -249,31 +312,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5;
 
   if (warp == kBwdLoadWarp) {
-    int uses[2] = {0, 0};
-    bool ok = true;
     if (ptx::elect_one()) {
       ptx::mbar_arrive_expect_tx(sm.fixed_full(), 2 * BwdCfg<D>::kTile);
       bwd_load_tile<D>(sm.fixed(0), &tm_k, sm.fixed_full(), kvh, k0 + kb * BN);
       bwd_load_tile<D>(sm.fixed(1), &tm_v, sm.fixed_full(), kvh, k0 + kb * BN);
     }
     __syncwarp();
-    for (int t = 0; t < n_tiles && ok; ++t) {
-      const int st = t & 1;
-      ok = __all_sync(FULL, wait_bar(sm.st_empty(st), ((t >> 1) & 1) ^ 1, ctl));
-      if (!ok) break;
-      ++uses[st];
-      const int h = kvh * G + t / per_head;
-      const int row = q0 + (qb0 + t % per_head) * BM;
-      if (ptx::elect_one()) {
-        ptx::mbar_arrive_expect_tx(sm.st_full(st), 2 * BwdCfg<D>::kTile);
-        bwd_load_tile<D>(sm.stage(st, 0), &tm_q, sm.st_full(st), h, row);
-        bwd_load_tile<D>(sm.stage(st, 1), &tm_do, sm.st_full(st), h, row);
-      }
-      __syncwarp();
-    }
+    bwd_stream<D>(sm, &tm_q, &tm_do, n_tiles, ctl, [&](int t, int& head, int& row) {
+      head = kvh * G + t / per_head;
+      row = q0 + (qb0 + t % per_head) * BM;
+    });
     drain_bar(sm.fixed_full(), 0);
-    for (int st = 0; st < 2; ++st)
-      if (uses[st] > 0) drain_bar(sm.st_full(st), (uses[st] - 1) & 1);
   } else if (warp == kBwdMmaWarp) {
     // Order per tile t: S^T(t), dP^T(t) | P(t) ready: dV(t), S^T(t+1) |
     // dS(t) ready: dK(t), dP^T(t+1). The compute warps turn S into P while
@@ -282,21 +331,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // (the tensor pipe runs in order).
     const uint64_t kd = desc_kmajor_sw128(ptx::smem_u32(sm.fixed(0)));
     const uint64_t vd = desc_kmajor_sw128(ptx::smem_u32(sm.fixed(1)));
+    using C = BwdCfg<D>;
     bool ok = __all_sync(FULL, wait_bar(sm.fixed_full(), 0, ctl));
-    auto stage_addr = [&](int t, int i) { return ptx::smem_u32(sm.stage(t & 1, i)); };
+    auto a_addr = [&](int t) { return ptx::smem_u32(sm.ring_a(ring_stage<C::kNA>(t))); };
+    auto b_addr = [&](int t) { return ptx::smem_u32(sm.ring_b(ring_stage<C::kNB>(t))); };
     auto issue_sT = [&](int t) {  // S^T(t) = K Q(t)^T
-      ok = __all_sync(FULL, wait_bar(sm.st_full(t & 1), (t >> 1) & 1, ctl));
+      ok = __all_sync(FULL, wait_bar(sm.a_full(ring_stage<C::kNA>(t)), ring_parity<C::kNA>(t), ctl));
       if (!ok) return;
       ptx::tc_fence_after();
       if (ptx::elect_one()) {
-        issue_s<D>(tmem + 0, kd, desc_kmajor_sw128(stage_addr(t, 0)));
+        issue_s<D>(tmem + 0, kd, desc_kmajor_sw128(a_addr(t)));
         ptx::tc_commit(sm.s_full());
       }
       __syncwarp();
     };
     auto issue_dpT = [&](int t) {  // dP^T(t) = V dO(t)^T
+      ok = __all_sync(FULL, wait_bar(sm.b_full(ring_stage<C::kNB>(t)), ring_parity<C::kNB>(t), ctl));
+      if (!ok) return;
+      ptx::tc_fence_after();
       if (ptx::elect_one()) {
-        issue_s<D>(tmem + 128, vd, desc_kmajor_sw128(stage_addr(t, 1)));
+        issue_s<D>(tmem + 128, vd, desc_kmajor_sw128(b_addr(t)));
         ptx::tc_commit(sm.dp_full());
       }
       __syncwarp();
@@ -309,10 +363,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(FULL, wait_bar(sm.p_full(), t & 1, ctl));
       if (!ok) break;
       ptx::tc_fence_after();
-      if (ptx::elect_one()) {  // dV += P^T dO
-        const uint64_t dmn = desc_mnmajor_sw128(stage_addr(t, 1), BwdCfg<D>::kChunk);
+      if (ptx::elect_one()) {  // dV += P^T dO; then dO(t)'s stage is free
+        const uint64_t dmn = desc_mnmajor_sw128(b_addr(t), BwdCfg<D>::kChunk);
         issue_pv_half<D>(tmem + 256, tmem + 0, dmn, 0, t > 0);
         issue_pv_half<D>(tmem + 256, tmem + 32, dmn, 1, true);  // rows 64.. at cols [64, 96)
+        ptx::tc_commit(sm.b_empty(ring_stage<C::kNB>(t)));
       }
       __syncwarp();
       if (t + 1 < n_tiles) {
@@ -322,11 +377,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(FULL, wait_bar(sm.ds_full(), t & 1, ctl));
       if (!ok) break;
       ptx::tc_fence_after();
-      if (ptx::elect_one()) {  // dK += dS^T Q
-        const uint64_t qmn = desc_mnmajor_sw128(stage_addr(t, 0), BwdCfg<D>::kChunk);
+      if (ptx::elect_one()) {  // dK += dS^T Q; then Q(t)'s stage is free
+        const uint64_t qmn = desc_mnmajor_sw128(a_addr(t), BwdCfg<D>::kChunk);
         issue_pv_half<D>(tmem + 256 + D, tmem + 128, qmn, 0, t > 0);
         issue_pv_half<D>(tmem + 256 + D, tmem + 160, qmn, 1, true);
-        ptx::tc_commit(sm.st_empty(t & 1));
+        ptx::tc_commit(sm.a_empty(ring_stage<C::kNA>(t)));
       }
       __syncwarp();
       if (t + 1 < n_tiles) issue_dpT(t + 1);
@@ -512,29 +567,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5;
 
   if (warp == kBwdLoadWarp) {
-    int uses[2] = {0, 0};
-    bool ok = true;
     if (n_k > 0 && ptx::elect_one()) {
       ptx::mbar_arrive_expect_tx(sm.fixed_full(), 2 * BwdCfg<D>::kTile);
       bwd_load_tile<D>(sm.fixed(0), &tm_q, sm.fixed_full(), h, q0 + qb * BM);
       bwd_load_tile<D>(sm.fixed(1), &tm_do, sm.fixed_full(), h, q0 + qb * BM);
     }
     __syncwarp();
-    for (int j = 0; j < n_k && ok; ++j) {
-      const int st = j & 1;
-      ok = __all_sync(FULL, wait_bar(sm.st_empty(st), ((j >> 1) & 1) ^ 1, ctl));
-      if (!ok) break;
-      ++uses[st];
-      if (ptx::elect_one()) {
-        ptx::mbar_arrive_expect_tx(sm.st_full(st), 2 * BwdCfg<D>::kTile);
-        bwd_load_tile<D>(sm.stage(st, 0), &tm_k, sm.st_full(st), kvh, k0 + j * BN);
-        bwd_load_tile<D>(sm.stage(st, 1), &tm_v, sm.st_full(st), kvh, k0 + j * BN);
-      }
-      __syncwarp();
-    }
+    bwd_stream<D>(sm, &tm_k, &tm_v, n_k, ctl, [&](int j, int& head, int& row) {
+      head = kvh;
+      row = k0 + j * BN;
+    });
     if (n_k > 0) drain_bar(sm.fixed_full(), 0);
-    for (int st = 0; st < 2; ++st)
-      if (uses[st] > 0) drain_bar(sm.st_full(st), (uses[st] - 1) & 1);
   } else if (warp == kBwdMmaWarp) {
     // Order per key tile j: S(j), dP(j) | S(j) read: S(j+1) | dS(j) ready:
     // dP(j+1), dQ(j). The compute warps turn S into P while dP(j) runs and
@@ -544,22 +587,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // which dQ(j) precedes.
     const uint64_t qd = desc_kmajor_sw128(ptx::smem_u32(sm.fixed(0)));
     const uint64_t dod = desc_kmajor_sw128(ptx::smem_u32(sm.fixed(1)));
+    using C = BwdCfg<D>;
     bool ok = n_k == 0 || __all_sync(FULL, wait_bar(sm.fixed_full(), 0, ctl));
-    auto stage_addr = [&](int j, int i) { return ptx::smem_u32(sm.stage(j & 1, i)); };
+    auto a_addr = [&](int j) { return ptx::smem_u32(sm.ring_a(ring_stage<C::kNA>(j))); };
+    auto b_addr = [&](int j) { return ptx::smem_u32(sm.ring_b(ring_stage<C::kNB>(j))); };
     auto issue_s_j = [&](int j) {  // S(j) = Q K(j)^T
-      ok = __all_sync(FULL, wait_bar(sm.st_full(j & 1), (j >> 1) & 1, ctl));
+      ok = __all_sync(FULL, wait_bar(sm.a_full(ring_stage<C::kNA>(j)), ring_parity<C::kNA>(j), ctl));
       if (!ok) return;
       ptx::tc_fence_after();
       if (ptx::elect_one()) {
-        issue_s<D>(tmem + 0, qd, desc_kmajor_sw128(stage_addr(j, 0)));
+        issue_s<D>(tmem + 0, qd, desc_kmajor_sw128(a_addr(j)));
         ptx::tc_commit(sm.s_full());
       }
       __syncwarp();
     };
-    auto issue_dp_j = [&](int j) {  // dP(j) = dO V(j)^T
+    auto issue_dp_j = [&](int j) {  // dP(j) = dO V(j)^T; then V(j)'s stage is free
+      ok = __all_sync(FULL, wait_bar(sm.b_full(ring_stage<C::kNB>(j)), ring_parity<C::kNB>(j), ctl));
+      if (!ok) return;
+      ptx::tc_fence_after();
       if (ptx::elect_one()) {
-        issue_s<D>(tmem + 128, dod, desc_kmajor_sw128(stage_addr(j, 1)));
+        issue_s<D>(tmem + 128, dod, desc_kmajor_sw128(b_addr(j)));
         ptx::tc_commit(sm.dp_full());
+        ptx::tc_commit(sm.b_empty(ring_stage<C::kNB>(j)));
       }
       __syncwarp();
     };
@@ -577,13 +626,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(FULL, wait_bar(sm.ds_full(), j & 1, ctl));
       if (!ok) break;
       ptx::tc_fence_after();
-      if (j + 1 < n_k) issue_dp_j(j + 1);
-      if (ptx::elect_one()) {  // dQ += dS K
-        const uint64_t kmn = desc_mnmajor_sw128(stage_addr(j, 0), BwdCfg<D>::kChunk);
+      if (j + 1 < n_k) {
+        issue_dp_j(j + 1);
+        if (!ok) break;
+      }
+      if (ptx::elect_one()) {  // dQ += dS K; then K(j)'s stage is free
+        const uint64_t kmn = desc_mnmajor_sw128(a_addr(j), BwdCfg<D>::kChunk);
         const uint32_t ds_col = tmem + 384 + 64 * (j & 1);
         issue_pv_half<D>(tmem + 256, ds_col, kmn, 0, j > 0);
         issue_pv_half<D>(tmem + 256, ds_col, kmn, 1, true);
-        ptx::tc_commit(sm.st_empty(j & 1));
+        ptx::tc_commit(sm.a_empty(ring_stage<C::kNA>(j)));
       }
       __syncwarp();
     }
