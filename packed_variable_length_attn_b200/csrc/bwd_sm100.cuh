@@ -58,13 +58,14 @@ struct BwdParams {
   int* error;
 };
 
-// Compute warps 0-7: warp w reads tensor-memory lanes 32(w % 4) .. +31 and
-// the half w / 4 of each 128-column tile (two warps per SM sub-partition).
-// MMA warp 8, load warp 9.
-constexpr int kBwdThreads = 320;
-constexpr int kBwdCompute = 256;
-constexpr int kBwdMmaWarp = 8;
-constexpr int kBwdLoadWarp = 9;
+// Compute warps 0-15: warp w reads tensor-memory lanes 32(w % 4) .. +31 and
+// the 32 columns 32(w / 4) .. +31 of each 128-column tile (four warps per SM
+// sub-partition, for latency hiding). MMA warp 16, load warp 17.
+constexpr int kBwdParts = 4;
+constexpr int kBwdCompute = 128 * kBwdParts;
+constexpr int kBwdThreads = kBwdCompute + 64;
+constexpr int kBwdMmaWarp = kBwdCompute / 32;
+constexpr int kBwdLoadWarp = kBwdMmaWarp + 1;
 
 // Stages of the two streamed-operand rings (see BwdCfg): 192 KB of shared
 // memory in all at head_dim 128, 160 KB at 64.
@@ -201,6 +202,19 @@ __device__ __forceinline__ void bwd_teardown(const BwdSmem<D>& sm, uint32_t tmem
   }
 }
 
+// D[tmem] (+)= A[tmem] * B[smem], K = 128 in steps of 16, with A written by
+// the four column parts: part p's 32 rows of K (bf16 pairs) sit in columns
+// a_base + 32p .. +15, i.e. K step k16 at a_base + 32(k16 / 2) + 8(k16 % 2).
+template <int D>
+__device__ __forceinline__ void issue_ts_parts(uint32_t d_tmem, uint32_t a_base, uint64_t b_desc,
+                                               bool acc) {
+  constexpr uint32_t idesc = idesc_bf16(D, true);
+#pragma unroll
+  for (int k16 = 0; k16 < 8; ++k16)
+    ptx::mma_ts(d_tmem, a_base + 32 * (k16 >> 1) + 8 * (k16 & 1),
+                b_desc + (uint64_t)((k16 * 16 * 128) >> 4), idesc, (acc || k16 > 0) ? 1u : 0u);
+}
+
 // Position of use u in a ring of N stages: stage and mbarrier parity.
 template <int N>
 __device__ __forceinline__ int ring_stage(int u) { return u % N; }
@@ -221,7 +235,6 @@ __device__ __forceinline__ void bwd_load_tile(uint8_t* dst, const CUtensorMap* t
 template <int C0, int C1>
 __device__ __forceinline__ void bwd_store_row(uint32_t t, bool have, float mul, __nv_bfloat16* dst,
                                               bool ok) {
-#pragma unroll
   for (int c = C0; c < C1; ++c) {
     uint32_t v[32];
     if (have) {
@@ -365,8 +378,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ptx::tc_fence_after();
       if (ptx::elect_one()) {  // dV += P^T dO; then dO(t)'s stage is free
         const uint64_t dmn = desc_mnmajor_sw128(b_addr(t), BwdCfg<D>::kChunk);
-        issue_pv_half<D>(tmem + 256, tmem + 0, dmn, 0, t > 0);
-        issue_pv_half<D>(tmem + 256, tmem + 32, dmn, 1, true);  // rows 64.. at cols [64, 96)
+        issue_ts_parts<D>(tmem + 256, tmem + 0, dmn, t > 0);
         ptx::tc_commit(sm.b_empty(ring_stage<C::kNB>(t)));
       }
       __syncwarp();
@@ -379,8 +391,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ptx::tc_fence_after();
       if (ptx::elect_one()) {  // dK += dS^T Q; then Q(t)'s stage is free
         const uint64_t qmn = desc_mnmajor_sw128(a_addr(t), BwdCfg<D>::kChunk);
-        issue_pv_half<D>(tmem + 256 + D, tmem + 128, qmn, 0, t > 0);
-        issue_pv_half<D>(tmem + 256 + D, tmem + 160, qmn, 1, true);
+        issue_ts_parts<D>(tmem + 256 + D, tmem + 128, qmn, t > 0);
         ptx::tc_commit(sm.a_empty(ring_stage<C::kNA>(t)));
       }
       __syncwarp();
@@ -390,10 +401,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
     drain_bar(sm.o_full(), 0);
   } else {
-    // compute warps: thread (c, hh) owns key kb*BN + c (tensor-memory lane c)
-    // and the query rows [64hh, 64hh + 64) of every tile
+    // compute warps: thread (c, part) owns key kb*BN + c (tensor-memory lane
+    // c) and the query rows [32 part, 32 part + 32) of every tile
     const int lane = threadIdx.x & 31;
-    const int c = (warp & 3) * 32 + lane, hh = warp >> 2, r0 = hh * 64;
+    const int c = (warp & 3) * 32 + lane, part = warp >> 2, r0 = part * 32;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t t_s = tmem + lane_base + r0, t_dp = tmem + lane_base + 128 + r0;
     const int kc = kb * BN + c;
@@ -407,11 +418,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         dbk = 0.f;
         if constexpr (kBiasKey) bkey = key_ok ? p.bias_key[(long long)(k0 + kc) * p.n_heads + h] : 0.f;
       }
-      // this tile's row constants: LSE * log2(e) and delta (written by the
-      // first 128 threads, read by all)
+      // this tile's row constants: LSE * log2(e) and delta (written by part
+      // 0, read by all)
       {
         const int b = t & 1;
-        if (hh == 0) {
+        if (part == 0) {
           const int rl = qb * BM + c;
           const long long gi = (long long)h * p.total_q + q0 + rl;
           sm.rows(b, 0)[c] = rl < Lq ? p.lse[gi] * kLog2e : 0.f;
@@ -425,8 +436,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       const float* lse2 = sm.rows(t & 1, 0);
       const float* dl = sm.rows(t & 1, 1);
-      // every row of this thread's half sees the key (no per-element mask)
-      const bool full = key_ok && qb * BM + r0 + 64 <= Lq && (!p.causal || kc <= qb * BM + r0 + off);
+      // every row of this thread's part sees the key (no per-element mask)
+      const bool full = key_ok && qb * BM + r0 + 32 <= Lq && (!p.causal || kc <= qb * BM + r0 + off);
       const float* grow = nullptr;
       if constexpr (kBiasPair)
         grow = p.bias_pair + (long long)seq * p.sb + (long long)(h / p.bias_head_div) * p.sh +
@@ -435,39 +446,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int ql = qb * BM + r;
         return key_ok && ql < Lq && (!p.causal || kc <= ql + off);
       };
-      // pass 1: S^T -> P^T, bf16 (to tensor memory for dV, over this half's
+      // pass 1: S^T -> P^T, bf16 (to tensor memory for dV, over this part's
       // own S^T columns, and kept packed in registers for dS)
       ok = __all_sync(FULL, wait_bar(sm.s_full(), t & 1, ctl));
       if (!ok) break;
       ptx::tc_fence_after();
-      uint32_t pk[32];
+      uint32_t pk[16];
       auto pass1 = [&](auto masked) {
-        uint32_t sv2[2][32];  // both chunks in flight before the first wait
-        ptx::tmem_ld32(t_s, sv2[0]);
-        ptx::tmem_ld32(t_s + 32, sv2[1]);
+        uint32_t sv[32];
+        ptx::tmem_ld32(t_s, sv);
         ptx::tmem_wait_ld();
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t (&sv)[32] = sv2[cc];
+        for (int e = 0; e < 32; e += 2) {
+          float pv[2];
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float pv[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int r = r0 + cc * 32 + e + u;
-              float x = __uint_as_float(sv[e + u]) * p.scale;
-              if constexpr (kBiasKey) x += bkey;
-              const bool vis = decltype(masked)::value ? visible(r) : true;
-              if constexpr (kBiasPair) {
-                if (vis) x += __ldg(grow + (long long)(qb * BM + r) * p.sr);
-              }
-              pv[u] = vis ? ptx::ex2(fmaf(x, kLog2e, -lse2[r])) : 0.f;
+          for (int u = 0; u < 2; ++u) {
+            const int r = r0 + e + u;
+            float x = __uint_as_float(sv[e + u]) * p.scale;
+            if constexpr (kBiasKey) x += bkey;
+            const bool vis = decltype(masked)::value ? visible(r) : true;
+            if constexpr (kBiasPair) {
+              if (vis) x += __ldg(grow + (long long)(qb * BM + r) * p.sr);
             }
-            pk[(cc * 32 + e) / 2] = ptx::pack_bf16x2(pv[0], pv[1]);
+            pv[u] = vis ? ptx::ex2(fmaf(x, kLog2e, -lse2[r])) : 0.f;
           }
-          // columns [r0 + 16cc, +16): this half's, already read
-          ptx::tmem_st16(t_s + cc * 16, &pk[cc * 16]);
+          pk[e / 2] = ptx::pack_bf16x2(pv[0], pv[1]);
         }
+        // columns [r0, r0 + 16): this part's, already read
+        ptx::tmem_st16(t_s, pk);
       };
       // (warp-uniform choice: the loop holds warp-collective tensor-memory
       // loads and stores)
@@ -484,42 +490,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                          ? nullptr
                          : p.dbias_pair + (long long)seq * p.dsb + (long long)h * p.dsh + kc;
       auto pass2 = [&](auto store_grid) {
-        uint32_t dp2[2][32];  // both chunks in flight before the first wait
-        ptx::tmem_ld32(t_dp, dp2[0]);
-        ptx::tmem_ld32(t_dp + 32, dp2[1]);
+        uint32_t dp[32];
+        ptx::tmem_ld32(t_dp, dp);
         ptx::tmem_wait_ld();
+        uint32_t dk16[16];
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t (&dp)[32] = dp2[cc];
-          uint32_t dk16[16];
+        for (int e = 0; e < 32; e += 2) {
+          const uint32_t w = pk[e / 2];
+          const float pv[2] = {__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)};
+          float dsv[2];
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const uint32_t w = pk[(cc * 32 + e) / 2];
-            const float pv[2] = {__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)};
-            float dsv[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int r = r0 + cc * 32 + e + u;
-              const float ds = pv[u] * (__uint_as_float(dp[e + u]) - dl[r]);
-              dbk += ds;
-              if constexpr (decltype(store_grid)::value) {
-                const int ql = qb * BM + r;
-                if (key_ok && ql < Lq) dgrow[(long long)ql * p.dsr] = ds;
-              }
-              dsv[u] = ds;
+          for (int u = 0; u < 2; ++u) {
+            const int r = r0 + e + u;
+            const float ds = pv[u] * (__uint_as_float(dp[e + u]) - dl[r]);
+            dbk += ds;
+            if constexpr (decltype(store_grid)::value) {
+              const int ql = qb * BM + r;
+              if (key_ok && ql < Lq) dgrow[(long long)ql * p.dsr] = ds;
             }
-            dk16[e / 2] = ptx::pack_bf16x2(dsv[0], dsv[1]);
+            dsv[u] = ds;
           }
-          ptx::tmem_st16(t_dp + cc * 16, dk16);
+          dk16[e / 2] = ptx::pack_bf16x2(dsv[0], dsv[1]);
         }
+        ptx::tmem_st16(t_dp, dk16);
       };
       if (dgrow != nullptr) pass2(std::true_type{});
       else pass2(std::false_type{});
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       ptx::mbar_arrive(sm.ds_full());
-      // two halves add into the zeroed output: 0 + a + b in either order is
-      // the same fp32 value, so the result stays deterministic
+      // the parts add into the zeroed output; the order of the adds is not
+      // fixed, so the per-key bias gradient can differ in the last bits
+      // between runs (dQ, dK, dV do not)
       if (p.dbias_key != nullptr && key_ok && t % per_head == per_head - 1)
         atomicAdd(p.dbias_key + (long long)(k0 + kc) * p.n_heads + h, dbk);
     }
@@ -528,14 +530,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = ok && __all_sync(FULL, wait_bar(sm.o_full(), 0, ctl));
       ptx::tc_fence_after();
     }
-    if (ok) {  // half 0 writes dV, half 1 dK
+    if (ok) {
+      // 2D/32 output chunks of 32 columns (dV's, then dK's) over the parts
       const long long o = ((long long)(k0 + kc) * p.n_kv_heads + kvh) * D;
-      if (hh == 0)
-        bwd_store_row<0, D / 32>(tmem + lane_base + 256, have, 1.f,
-                                 reinterpret_cast<__nv_bfloat16*>(p.dv) + o, key_ok);
-      else
-        bwd_store_row<0, D / 32>(tmem + lane_base + 256 + D, have, p.scale,
-                                 reinterpret_cast<__nv_bfloat16*>(p.dk) + o, key_ok);
+      constexpr int kCh = D / 32;
+      for (int q = part; q < 2 * kCh; q += kBwdParts) {
+        const bool is_k = q >= kCh;
+        const int ch = is_k ? q - kCh : q;
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(is_k ? p.dk : p.dv) + o;
+        bwd_store_row<0, 1>(tmem + lane_base + 256 + (is_k ? D : 0) + ch * 32, have,
+                            is_k ? p.scale : 1.f, dst + ch * 32, key_ok);
+      }
     }
   }
   bwd_teardown<D>(sm, tmem);
@@ -643,10 +648,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
     drain_bar(sm.o_full(), 0);
   } else {
-    // compute warps: thread (r, hh) owns query row qb*BM + r and the keys
-    // [64hh, 64hh + 64) of every tile
+    // compute warps: thread (r, part) owns query row qb*BM + r and the keys
+    // [32 part, 32 part + 32) of every tile
     const int lane = threadIdx.x & 31;
-    const int r = (warp & 3) * 32 + lane, hh = warp >> 2, c0 = hh * 64;
+    const int r = (warp & 3) * 32 + lane, part = warp >> 2, c0 = part * 32;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t t_s = tmem + lane_base + c0, t_dp = tmem + lane_base + 128 + c0;
     const int ql = qb * BM + r;
@@ -660,36 +665,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
              (long long)ql * p.sr;
     bool ok = true;
     for (int j = 0; j < n_k && ok; ++j) {
-      const int kt = j * BN + c0;  // this half's first key
-      // every key of this half is visible to the row (no per-element mask)
-      const bool full = row_ok && kt + 64 <= Lk && (!p.causal || kt + 63 <= ql + off);
+      const int kt = j * BN + c0;  // this part's first key
+      // every key of this part is visible to the row (no per-element mask)
+      const bool full = row_ok && kt + 32 <= Lk && (!p.causal || kt + 31 <= ql + off);
       ok = __all_sync(FULL, wait_bar(sm.s_full(), j & 1, ctl));
       if (!ok) break;
       ptx::tc_fence_after();
-      float pr[64];
+      float pr[32];
       auto pass1 = [&](auto masked) {
-        uint32_t sv2[2][32];  // both chunks in flight before the first wait
-        ptx::tmem_ld32(t_s, sv2[0]);
-        ptx::tmem_ld32(t_s + 32, sv2[1]);
+        uint32_t sv[32];
+        ptx::tmem_ld32(t_s, sv);
         ptx::tmem_wait_ld();
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t (&sv)[32] = sv2[cc];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int kc = kt + cc * 32 + e;
-            const bool vis = decltype(masked)::value
-                                 ? row_ok && kc < Lk && (!p.causal || kc <= ql + off)
-                                 : true;
-            float x = __uint_as_float(sv[e]) * p.scale;
-            if constexpr (kBiasKey) {
-              if (vis) x += __ldg(p.bias_key + (long long)(k0 + kc) * p.n_heads + h);
-            }
-            if constexpr (kBiasPair) {
-              if (vis) x += __ldg(grow + (long long)kc * p.sc);
-            }
-            pr[cc * 32 + e] = vis ? ptx::ex2(fmaf(x, kLog2e, -lse2)) : 0.f;
+        for (int e = 0; e < 32; ++e) {
+          const int kc = kt + e;
+          const bool vis = decltype(masked)::value
+                               ? row_ok && kc < Lk && (!p.causal || kc <= ql + off)
+                               : true;
+          float x = __uint_as_float(sv[e]) * p.scale;
+          if constexpr (kBiasKey) {
+            if (vis) x += __ldg(p.bias_key + (long long)(k0 + kc) * p.n_heads + h);
           }
+          if constexpr (kBiasPair) {
+            if (vis) x += __ldg(grow + (long long)kc * p.sc);
+          }
+          pr[e] = vis ? ptx::ex2(fmaf(x, kLog2e, -lse2)) : 0.f;
         }
       };
       // (warp-uniform choice: the loop holds warp-collective loads)
@@ -700,19 +700,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(FULL, wait_bar(sm.dp_full(), j & 1, ctl));
       if (!ok) break;
       ptx::tc_fence_after();
-      uint32_t dp2[2][32];  // both chunks in flight before the first wait
-      ptx::tmem_ld32(t_dp, dp2[0]);
-      ptx::tmem_ld32(t_dp + 32, dp2[1]);
-      ptx::tmem_wait_ld();
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t (&dp)[32] = dp2[cc];
+      {
+        uint32_t dp[32];
+        ptx::tmem_ld32(t_dp, dp);
+        ptx::tmem_wait_ld();
         uint32_t dk16[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2)
-          dk16[e / 2] = ptx::pack_bf16x2(pr[cc * 32 + e] * (__uint_as_float(dp[e]) - dl),
-                                         pr[cc * 32 + e + 1] * (__uint_as_float(dp[e + 1]) - dl));
-        ptx::tmem_st16(tmem + lane_base + 384 + 64 * (j & 1) + hh * 32 + cc * 16, dk16);
+          dk16[e / 2] = ptx::pack_bf16x2(pr[e] * (__uint_as_float(dp[e]) - dl),
+                                         pr[e + 1] * (__uint_as_float(dp[e + 1]) - dl));
+        // dS(j) buffer j % 2: this part's 32 keys in columns [16 part, +16)
+        ptx::tmem_st16(tmem + lane_base + 384 + 64 * (j & 1) + 16 * part, dk16);
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
@@ -723,13 +721,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = ok && __all_sync(FULL, wait_bar(sm.o_full(), 0, ctl));
       ptx::tc_fence_after();
     }
-    if (ok) {  // half hh writes columns [hh * D/2, (hh + 1) * D/2) of the row
+    if (ok) {  // D/32 output chunks of 32 columns over the parts
       __nv_bfloat16* dst =
           reinterpret_cast<__nv_bfloat16*>(p.dq) + ((long long)(q0 + ql) * p.n_heads + h) * D;
-      if (hh == 0)
-        bwd_store_row<0, D / 64>(tmem + lane_base + 256, have, p.scale, dst, row_ok);
-      else
-        bwd_store_row<D / 64, D / 32>(tmem + lane_base + 256, have, p.scale, dst, row_ok);
+      for (int ch = part; ch < D / 32; ch += kBwdParts)
+        bwd_store_row<0, 1>(tmem + lane_base + 256 + ch * 32, have, p.scale, dst + ch * 32, row_ok);
     }
   }
   bwd_teardown<D>(sm, tmem);

@@ -101,6 +101,39 @@ def test_backward_with_biases(causal):
     _run([33, 150, 1, 200], [40, 150, 17, 260], 4, 2, 64, causal, seed=91 + causal, bias=True)
 
 
+def test_backward_broadcast_and_strided_grid():
+    # one grid shared by all heads (head stride 0), read through a permuted
+    # view (column stride != 1: the per-element load path)
+    lq, lk = [60, 131], [70, 131]
+    Hq, Hkv, D = 4, 2, 64
+    w = workloads.make_custom(lq, lk, n_heads=Hq, n_kv_heads=Hkv, head_dim=D, causal=True,
+                              seed=211)
+    g = torch.Generator().manual_seed(212)
+    base = torch.randn(len(lq), max(lk), max(lq), generator=g)   # [B, C, R]
+    grid = base.permute(0, 2, 1)                                  # [B, R, C] view, sc = R
+    strides = (grid.stride(0), 0, grid.stride(1), grid.stride(2))
+    dev = to_device(w)
+    kw = dict(softmax_scale=w.softmax_scale, causal=True, bias_pair=base.cuda().permute(0, 2, 1),
+              bias_pair_strides=strides)
+    out, lse = va.varlen_attn_fwd(dev["q"], dev["k"], dev["v"], dev["cu_q"], dev["cu_k"],
+                                  w.max_seqlen_q, w.max_seqlen_k, **kw)
+    dout = torch.randn(w.q.shape, generator=g).to(torch.bfloat16)
+    dq, dk, dv, _, dbp = va.varlen_attn_bwd(dev["q"], dev["k"], dev["v"], out, lse, dout.cuda(),
+                                            dev["cu_q"], dev["cu_k"], w.max_seqlen_q,
+                                            w.max_seqlen_k, need_dbias_pair=True, **kw)
+    torch.cuda.synchronize()
+    flat = base.contiguous()  # the oracle reads the same entries through the same strides
+    ref = oracle_bwd(w.q, w.k, w.v, dout, w.cu_q, w.cu_k, Hq, Hkv, w.softmax_scale, True,
+                     bias_pair=flat, bias_strides=strides)
+    _close("dq", dq.float().cpu().numpy(), ref["dq"])
+    _close("dk", dk.float().cpu().numpy(), ref["dk"])
+    _close("dv", dv.float().cpu().numpy(), ref["dv"])
+    _close("dbias_pair", dbp.cpu().numpy(), ref["dbias_pair"])
+    # the broadcast grid's own gradient is the sum over the heads
+    _close("dbias_pair summed over heads", dbp.sum(dim=1).cpu().numpy(),
+           ref["dbias_pair"].sum(axis=1))
+
+
 def test_backward_kv_head_grid():
     _run([50, 140], [60, 140], 4, 2, 64, True, seed=123, bias=True, kv_head_grid=True)
 
