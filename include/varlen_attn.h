@@ -226,11 +226,14 @@ int varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v,
  *   h*dbias_stride_h + r*dbias_stride_q + c for every query head h and every
  *   in-sequence (r, c); other entries are left as they are. A broadcast or
  *   per-K/V-head grid's gradient is the sum of these over the heads that read it.
- * Rows without a visible key get zero gradients. Deterministic (no atomics):
- * one launch validates cu_seqlens (a bad table raises VARLEN_ATTN_ERR_BAD_SEQLENS
- * on the device and writes no gradient), one computes delta into the library
- * workspace, one computes dK and dV per (sequence, K/V head, 128-key block),
- * one dQ per (sequence, query head, 128-row block). Errors as for
+ * Rows without a visible key get zero gradients. dq, dk, dv and dbias_pair
+ * are bitwise reproducible (no atomics); dbias_per_key is the sum of four
+ * partial sums added atomically into the zeroed buffer, so its last bits may
+ * vary between runs. Launches: one validates cu_seqlens (a bad table raises
+ * VARLEN_ATTN_ERR_BAD_SEQLENS on the device and writes no gradient), one
+ * computes delta into the library workspace, one computes dK and dV per
+ * (sequence, K/V head, 128-key block), one dQ per (sequence, query head,
+ * 128-row block); with dbias_per_key a memset zeroes it first. Errors as for
  * varlen_attn_fwd; batch or n_heads above 65535: VARLEN_ATTN_ERR_TOO_LARGE.
  */
 int varlen_attn_bwd(const void* q, const void* k, const void* v, const void* out,
