@@ -1,6 +1,7 @@
 /*
- * varlen_attn.h — C ABI of the packed variable-length attention forward
- * library for NVIDIA B200 (sm_100a). Link: libvarlen_attn.so.
+ * varlen_attn.h — C ABI of the packed variable-length attention library for
+ * NVIDIA B200 (sm_100a): the forward, its backward, a K/V-cache decode step
+ * and the packed-layout helpers. Link: libvarlen_attn.so.
  *
  * The operation (pages cited by title and section):
  *   Many ragged sequences are concatenated into one token stream; explicit
