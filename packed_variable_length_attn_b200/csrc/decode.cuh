@@ -19,6 +19,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace va {
 
@@ -158,9 +159,11 @@ __global__ void __launch_bounds__(kDecThreads, RT <= 8 ? 4 : 2) decode_kernel(De
     l_s[rho] = 0.f;
   }
   const int dp = tid % kNPair, kg = tid / kNPair;  // P V: dims 2dp, 2dp+1; key group kg
-  float acc[RT][2];
+  // O accumulators: dims 2dp and 2dp + 1 of the row pairs (2i, 2i + 1), as
+  // packed fp32 pairs (one packed FMA updates two rows)
+  uint64_t ax[RT / 2], ay[RT / 2];
 #pragma unroll
-  for (int rho = 0; rho < RT; ++rho) acc[rho][0] = acc[rho][1] = 0.f;
+  for (int i = 0; i < RT / 2; ++i) ax[i] = ay[i] = 0ull;
 
   const long long row_stride = (long long)p.n_kv_heads * D;  // elements between cache rows
   const __nv_bfloat16* kbase = p.k_cache + (long long)i * p.cache_len * row_stride + (long long)g * D;
@@ -202,14 +205,12 @@ __global__ void __launch_bounds__(kDecThreads, RT <= 8 ? 4 : 2) decode_kernel(De
 #pragma unroll
     for (int pass = 0; pass < kDecKeys / kKPP; ++pass) {
       const int kr = pass * kKPP + tid / kTPK, c = tid % kTPK;
-      float kf[kDPT];
+      uint64_t kf[kDPT / 2];  // dim pairs (4c + 32m, +1) and (+2, +3)
 #pragma unroll
       for (int m = 0; m < D / 32; ++m) {
         const uint2 raw = *reinterpret_cast<const uint2*>(kb + kr * S::kKS + 32 * m + 4 * c);
-        kf[4 * m] = bf16_lo(raw.x);
-        kf[4 * m + 1] = bf16_hi(raw.x);
-        kf[4 * m + 2] = bf16_lo(raw.y);
-        kf[4 * m + 3] = bf16_hi(raw.y);
+        kf[2 * m] = ptx::f2(bf16_lo(raw.x), bf16_hi(raw.x));
+        kf[2 * m + 1] = ptx::f2(bf16_lo(raw.y), bf16_hi(raw.y));
       }
       const int key = k0 + kr;
 #pragma unroll 1
@@ -218,15 +219,15 @@ __global__ void __launch_bounds__(kDecThreads, RT <= 8 ? 4 : 2) decode_kernel(De
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float* qrow = qs + (r0 + j) * D + 4 * c;
-          float a = 0.f, b = 0.f;
+          uint64_t ab = 0ull;  // even dims | odd dims
 #pragma unroll
           for (int m = 0; m < D / 32; ++m) {
-            const float4 qv = *reinterpret_cast<const float4*>(qrow + 32 * m);
-            a = fmaf(qv.x, kf[4 * m], a);
-            b = fmaf(qv.y, kf[4 * m + 1], b);
-            a = fmaf(qv.z, kf[4 * m + 2], a);
-            b = fmaf(qv.w, kf[4 * m + 3], b);
+            const ulonglong2 qv = *reinterpret_cast<const ulonglong2*>(qrow + 32 * m);
+            ab = ptx::ffma2(qv.x, kf[2 * m], ab);
+            ab = ptx::ffma2(qv.y, kf[2 * m + 1], ab);
           }
+          float a, b;
+          ptx::f2_split(ab, a, b);
           part[j] = a + b;
         }
 #pragma unroll
@@ -274,28 +275,25 @@ __global__ void __launch_bounds__(kDecThreads, RT <= 8 ? 4 : 2) decode_kernel(De
     __syncthreads();
     // O = O * fac + P V over this thread's key group
 #pragma unroll
-    for (int rho = 0; rho < RT; ++rho) {
-      const float f = f_s[rho];
-      acc[rho][0] *= f;
-      acc[rho][1] *= f;
+    for (int i = 0; i < RT / 2; ++i) {
+      const uint64_t f = *reinterpret_cast<const uint64_t*>(f_s + 2 * i);
+      ax[i] = ptx::ffma2(ax[i], f, 0ull);
+      ay[i] = ptx::ffma2(ay[i], f, 0ull);
     }
 #pragma unroll 4
     for (int kk = 0; kk < kKPG; ++kk) {
       const int key = kg * kKPG + kk;
       const uint32_t vraw = *reinterpret_cast<const uint32_t*>(vb + key * S::kKS + 2 * dp);
-      const float2 v = make_float2(bf16_lo(vraw), bf16_hi(vraw));
-      const float4* prow = reinterpret_cast<const float4*>(ps + key * RT);
+      const float vx = bf16_lo(vraw), vy = bf16_hi(vraw);
+      const uint64_t vx2 = ptx::f2(vx, vx), vy2 = ptx::f2(vy, vy);
+      const ulonglong2* prow = reinterpret_cast<const ulonglong2*>(ps + key * RT);
 #pragma unroll
       for (int r4 = 0; r4 < RT / 4; ++r4) {
-        const float4 pv = prow[r4];
-        acc[4 * r4][0] = fmaf(pv.x, v.x, acc[4 * r4][0]);
-        acc[4 * r4][1] = fmaf(pv.x, v.y, acc[4 * r4][1]);
-        acc[4 * r4 + 1][0] = fmaf(pv.y, v.x, acc[4 * r4 + 1][0]);
-        acc[4 * r4 + 1][1] = fmaf(pv.y, v.y, acc[4 * r4 + 1][1]);
-        acc[4 * r4 + 2][0] = fmaf(pv.z, v.x, acc[4 * r4 + 2][0]);
-        acc[4 * r4 + 2][1] = fmaf(pv.z, v.y, acc[4 * r4 + 2][1]);
-        acc[4 * r4 + 3][0] = fmaf(pv.w, v.x, acc[4 * r4 + 3][0]);
-        acc[4 * r4 + 3][1] = fmaf(pv.w, v.y, acc[4 * r4 + 3][1]);
+        const ulonglong2 pp = prow[r4];  // rows (4r4, 4r4 + 1) | (4r4 + 2, 4r4 + 3)
+        ax[2 * r4] = ptx::ffma2(pp.x, vx2, ax[2 * r4]);
+        ay[2 * r4] = ptx::ffma2(pp.x, vy2, ay[2 * r4]);
+        ax[2 * r4 + 1] = ptx::ffma2(pp.y, vx2, ax[2 * r4 + 1]);
+        ay[2 * r4 + 1] = ptx::ffma2(pp.y, vy2, ay[2 * r4 + 1]);
       }
     }
     __syncthreads();  // this stage is reloaded by the next iteration; ps, f_s reused
@@ -309,10 +307,16 @@ __global__ void __launch_bounds__(kDecThreads, RT <= 8 ? 4 : 2) decode_kernel(De
   for (int grp = 0; grp < kNKG; ++grp) {
     if (kg == grp) {
 #pragma unroll
-      for (int rho = 0; rho < RT; ++rho) {
-        float2* dst = reinterpret_cast<float2*>(osum + rho * D + 2 * dp);
-        const float2 prev = grp == 0 ? make_float2(0.f, 0.f) : *dst;
-        *dst = make_float2(prev.x + acc[rho][0], prev.y + acc[rho][1]);
+      for (int i = 0; i < RT / 2; ++i) {
+        float x0, x1, y0, y1;
+        ptx::f2_split(ax[i], x0, x1);
+        ptx::f2_split(ay[i], y0, y1);
+        float2* d0 = reinterpret_cast<float2*>(osum + (2 * i) * D + 2 * dp);
+        float2* d1 = reinterpret_cast<float2*>(osum + (2 * i + 1) * D + 2 * dp);
+        const float2 p0 = grp == 0 ? make_float2(0.f, 0.f) : *d0;
+        const float2 p1 = grp == 0 ? make_float2(0.f, 0.f) : *d1;
+        *d0 = make_float2(p0.x + x0, p0.y + y0);
+        *d1 = make_float2(p1.x + x1, p1.y + y1);
       }
     }
     __syncthreads();
