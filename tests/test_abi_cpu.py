@@ -163,3 +163,19 @@ def test_backward_host_validation_codes(lib):
     assert call(dbp=16, dsb=-1) == 6
     assert call(flags=2) == 6
     assert call(batch=70000) == 11
+
+
+def test_backward_binding_rejects_bad_tensors(lib):
+    q = torch.zeros(4, 2, 64, dtype=torch.bfloat16)
+    k = torch.zeros(4, 1, 64, dtype=torch.bfloat16)
+    lse = torch.zeros(2, 4)
+    cu = torch.tensor([0, 4], dtype=torch.int32)
+    # host tensors: the binding refuses them (no CPU path)
+    with pytest.raises(ValueError):
+        va.varlen_attn_bwd(q, k, k, q, lse, q, cu, cu, 4, 4)
+    # wrong dtype
+    with pytest.raises(ValueError):
+        va.varlen_attn_bwd(q.float(), k, k, q, lse, q, cu, cu, 4, 4)
+    # dout of the wrong shape
+    with pytest.raises(ValueError):
+        va.varlen_attn_bwd(q, k, k, q, lse, q[:2], cu, cu, 4, 4)
