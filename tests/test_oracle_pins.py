@@ -12,6 +12,7 @@ import os
 
 import numpy as np
 import pytest
+from hypothesis import HealthCheck, given, settings, strategies as st
 import torch
 
 import oracle
@@ -313,3 +314,33 @@ def test_oracle_rejects_malformed_arguments():
     bad[2] = 1  # decreasing boundaries
     with pytest.raises(ValueError):
         oracle.fwd(w.q, w.k, w.v, bad, w.cu_k, 2, 2, w.softmax_scale, True)
+
+
+# --------------------------------------------------------------------------- randomized brute force
+
+
+@settings(max_examples=40, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(data=st.data())
+def test_oracle_matches_bruteforce_random_shapes(data):
+    """Random packs (empty members, Lq != Lk, GQA groups, both biases) against
+    the padded brute force: any index or mask slip in either shows here."""
+    B = data.draw(st.integers(1, 4))
+    lq = data.draw(st.lists(st.integers(0, 12), min_size=B, max_size=B))
+    lk = data.draw(st.lists(st.integers(0, 12), min_size=B, max_size=B))
+    hkv = data.draw(st.sampled_from([1, 2]))
+    g = data.draw(st.sampled_from([1, 2, 3]))
+    D = data.draw(st.sampled_from([4, 8]))
+    causal = data.draw(st.booleans())
+    bias = data.draw(st.sampled_from(["none", "key", "pair", "both"]))
+    seed = data.draw(st.integers(0, 10_000))
+    if sum(lq) == 0:
+        lq[0] = 1
+    mq, mk = max(max(lq), 1), max(max(lk), 1)
+    w = workloads.make_custom(lq, lk, n_heads=hkv * g, n_kv_heads=hkv, head_dim=D,
+                              causal=causal, seed=seed, bias_key=bias in ("key", "both"),
+                              bias_pair=(B, hkv * g, mq, mk) if bias in ("pair", "both") else None)
+    out, lse = _run_oracle(w)
+    bo, bl = padded_attention(w.q, w.k, w.v, w.cu_q, w.cu_k, w.n_heads, w.n_kv_heads,
+                              w.softmax_scale, w.causal, w.bias_key, w.bias_pair, w.bias_strides)
+    np.testing.assert_allclose(out, bo, rtol=0, atol=1e-12)
+    _assert_close_inf(lse, bl, 1e-12)
