@@ -13,6 +13,7 @@
 """
 import numpy as np
 import pytest
+from hypothesis import HealthCheck, given, settings, strategies as st
 
 import oracle
 from oracle.backward import bwd
@@ -121,3 +122,43 @@ def test_single_key_sequence():
     g = bwd(q, k, v, dout, [0, 3], [0, 1], 2, 2, 0.5, False)
     assert np.abs(g["dq"]).max() == 0.0 and np.abs(g["dk"]).max() == 0.0
     np.testing.assert_allclose(g["dv"][0], dout.sum(axis=0), rtol=1e-14)
+
+
+@settings(max_examples=15, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(data=st.data())
+def test_finite_differences_random_packs(data):
+    """Random packs (empty members, Lq != Lk, GQA, biases): sampled gradient
+    entries against central differences of the forward oracle."""
+    B = data.draw(st.integers(1, 3))
+    lq = data.draw(st.lists(st.integers(0, 6), min_size=B, max_size=B))
+    lk = data.draw(st.lists(st.integers(1, 6), min_size=B, max_size=B))
+    if sum(lq) == 0:
+        lq[0] = 1
+    hkv = data.draw(st.sampled_from([1, 2]))
+    Hq = hkv * data.draw(st.sampled_from([1, 2]))
+    D = 4
+    causal = data.draw(st.booleans())
+    with_bias = data.draw(st.booleans())
+    rng = np.random.default_rng(data.draw(st.integers(0, 10_000)))
+    cu_q = np.concatenate([[0], np.cumsum(lq)]).astype(np.int32)
+    cu_k = np.concatenate([[0], np.cumsum(lk)]).astype(np.int32)
+    c = dict(q=rng.standard_normal((int(cu_q[-1]), Hq, D)),
+             k=rng.standard_normal((int(cu_k[-1]), hkv, D)),
+             v=rng.standard_normal((int(cu_k[-1]), hkv, D)),
+             dout=rng.standard_normal((int(cu_q[-1]), Hq, D)),
+             cu_q=cu_q, cu_k=cu_k, Hq=Hq, Hkv=hkv, scale=0.41, causal=causal,
+             bk=None, bp=None, strides=None)
+    if with_bias:
+        R, C = max(max(lq), 1), max(lk)
+        c["bk"] = rng.standard_normal((int(cu_k[-1]), Hq)) * 0.5
+        c["bp"] = rng.standard_normal((B, Hq, R, C))
+        c["strides"] = (Hq * R * C, R * C, C, 1)
+    g = _grads(c)
+    h = 1e-5
+    for name, key in (("q", "dq"), ("k", "dk"), ("v", "dv")) + ((("bk", "dbias_key"),) if with_bias else ()):
+        x = c[name]
+        idx = tuple(int(rng.integers(0, s)) for s in x.shape)
+        xp = x.copy(); xp[idx] += h
+        xm = x.copy(); xm[idx] -= h
+        fd = (_loss(c, **{name: xp}) - _loss(c, **{name: xm})) / (2 * h)
+        assert abs(g[key][idx] - fd) <= 1e-6 * (1 + abs(fd)), (name, idx, g[key][idx], fd)
