@@ -9,25 +9,29 @@
 // backward, and the ASpec PR 25 page, "Verification", bounds Q/K/V gradient
 // errors at 1% relative L2 against a dense math backend).
 //
-// Two kernels, each deterministic (no atomics), one CTA per SM:
+// Two kernels, one CTA per SM; dQ, dK and dV are computed without atomics,
+// so they do not depend on scheduling:
 //   attn_bwd_dkdv_sm100: one CTA per (sequence, K/V head, 128-key block).
 //     K and V stay in shared memory; for every query head of the group and
 //     every 128-row query block that can see the keys, Q and dO arrive by
-//     TMA (two stages) and the tensor cores compute
+//     TMA (a ring each) and the tensor cores compute
 //       S^T  = K Q^T       (tensor memory cols [0,128): keys are the lanes)
 //       dP^T = V dO^T      (cols [128,256))
-//     the four compute warps turn them into P^T and dS^T (bf16, written
-//     back over S^T and dP^T), and
+//     the sixteen compute warps (four per lane quarter, 32 columns each)
+//     turn them into P^T and dS^T (bf16, written back over each part's own
+//     S^T and dP^T columns), and
 //       dV  += P^T dO      (cols [256, 256+D), P^T read from tensor memory)
 //       dK  += dS^T Q      (cols [256+D, 256+2D))
 //     Each thread owns one key, so the per-key bias gradient is a register
-//     sum and the pair-grid gradient rows are written coalesced.
+//     sum per part (the four parts add atomically) and the pair-grid gradient
+//     rows are written coalesced.
 //   attn_bwd_dq_sm100: one CTA per (sequence, query head, 128-row block).
-//     Q and dO stay; K and V stream in two stages; S = Q K^T, dP = dO V^T,
-//     dS as above (one thread per query row), dQ += dS K.
+//     Q and dO stay; K and V stream in rings of their own; S = Q K^T,
+//     dP = dO V^T, dS as above (one thread per query row and column part),
+//     dQ += dS K.
 // The pair of kernels recomputes S and dP once more than a single fused
-// kernel with atomic dQ accumulation would; in exchange nothing is reduced
-// across CTAs and the results do not depend on scheduling.
+// kernel with atomic dQ accumulation would; in exchange nothing of Q, K, V's
+// gradients is reduced across CTAs.
 #pragma once
 #include <type_traits>
 
