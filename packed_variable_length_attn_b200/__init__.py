@@ -1,4 +1,4 @@
-"""Packed variable-length attention forward for NVIDIA B200 (sm_100a).
+"""Packed variable-length attention for NVIDIA B200 (sm_100a).
 
 Thin Python binding over the C ABI of ``libvarlen_attn.so`` (declared in
 ``include/varlen_attn.h``). This module only checks and marshals arguments:
@@ -13,6 +13,16 @@ library is missing or the device is not sm_100, calls raise.
 ``[total_k, n_kv_heads, head_dim]`` (bf16, or fp32 for the fp32 path),
 ``cu_seqlens_*`` are int32 ``[batch + 1]`` on the same device. ``out`` has
 q's shape and dtype; ``lse`` is fp32 ``[n_heads, total_q]``.
+
+Also: ``varlen_attn_bwd`` (gradients of q, k, v and the biases from the
+forward's ``out`` and ``lse`` and the output gradient), ``varlen_attn_decode``
+(a decode step over a per-sequence K/V cache), ``unpad`` / ``pad`` /
+``mask_to_seqlens`` / ``gather_rows`` / ``scatter_rows`` (packed-layout
+helpers) and ``fold_pair_bias_row`` (first-token bias fold).
+
+    dq, dk, dv, _, _ = varlen_attn_bwd(q, k, v, out, lse, dout, cu_seqlens_q,
+                                       cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                                       causal=True)
 """
 from __future__ import annotations
 
