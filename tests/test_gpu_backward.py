@@ -148,3 +148,34 @@ def test_backward_deterministic():
     b = _run([200, 77], [260, 77], 4, 2, 128, True, seed=17)
     for x, y in zip(a, b):
         assert torch.equal(x.view(torch.int16), y.view(torch.int16))
+
+
+def test_backward_packed_equals_solo_bit_exact():
+    # each sequence's gradients, run alone, equal its slice of the packed run
+    # bit for bit (the other sequences contribute exact zeros)
+    lq, lk = [150, 7, 260], [170, 40, 260]
+    Hq, Hkv, D = 4, 2, 128
+    w = workloads.make_custom(lq, lk, n_heads=Hq, n_kv_heads=Hkv, head_dim=D, causal=True,
+                              seed=404)
+    g = torch.Generator().manual_seed(405)
+    dout = torch.randn(w.q.shape, generator=g).to(torch.bfloat16)
+    dev = to_device(w)
+    kw = dict(softmax_scale=w.softmax_scale, causal=True)
+    out, lse = va.varlen_attn_fwd(dev["q"], dev["k"], dev["v"], dev["cu_q"], dev["cu_k"],
+                                  w.max_seqlen_q, w.max_seqlen_k, **kw)
+    dq, dk, dv, _, _ = va.varlen_attn_bwd(dev["q"], dev["k"], dev["v"], out, lse, dout.cuda(),
+                                          dev["cu_q"], dev["cu_k"], w.max_seqlen_q,
+                                          w.max_seqlen_k, **kw)
+    cq, ck = w.cu_q.tolist(), w.cu_k.tolist()
+    for i in range(len(lq)):
+        qs, ks = slice(cq[i], cq[i + 1]), slice(ck[i], ck[i + 1])
+        one = lambda n: torch.tensor([0, n], dtype=torch.int32, device="cuda")
+        q1, k1, v1 = (dev["q"][qs].contiguous(), dev["k"][ks].contiguous(),
+                      dev["v"][ks].contiguous())
+        o1, l1 = va.varlen_attn_fwd(q1, k1, v1, one(lq[i]), one(lk[i]), lq[i], lk[i], **kw)
+        d1 = va.varlen_attn_bwd(q1, k1, v1, o1, l1, dout[qs].contiguous().cuda(), one(lq[i]),
+                                one(lk[i]), lq[i], lk[i], **kw)
+        torch.cuda.synchronize()
+        assert torch.equal(d1[0].view(torch.int16), dq[qs].view(torch.int16)), i
+        assert torch.equal(d1[1].view(torch.int16), dk[ks].view(torch.int16)), i
+        assert torch.equal(d1[2].view(torch.int16), dv[ks].view(torch.int16)), i
