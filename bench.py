@@ -44,8 +44,14 @@ BIAS = {3: "pair grid fp32 [512,1,256,256] N(0,1), strides (65536,0,256,1); "
            "per-key fp32 [Tk,8] N(0,0.5)"}
 L2_SCRUB_BYTES = 256 << 20
 KERNEL_SOURCES = ["attn_sm100.cuh", "ptx.cuh", "common.cuh"]
-PROFILE_FILE = os.path.join(ROOT, "profiles", "attn_fwd_sm100_long_causal_gqa.md")
+PROFILE_FILE = os.path.join(ROOT, "profiles", "attn_fwd_sm100_long_causal_gqa.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# NVIDIA's datasheet dense BF16 tensor figure for one B200: the HGX B200
+# datasheet lists 36 PFLOPS FP16/BF16 per 8 GPUs with 2:4 sparsity, i.e.
+# 18 PFLOPS dense per 8 GPUs = 2.25 PFLOPS per GPU.
+DATASHEET_BF16_TFLOPS = 2250.0
+DATASHEET_SOURCE = ("NVIDIA HGX B200 datasheet: 36 PFLOPS FP16/BF16 per 8 GPUs with 2:4 "
+                    "sparsity = 2.25 PFLOPS dense per GPU")
 
 
 def _peaks():
@@ -66,57 +72,120 @@ def kernel_source_hash() -> str:
 
 
 def _profiled_traffic():
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source; else None."""
+    """DRAM bytes per launch of the attention kernel on the full long
+    workload, from the committed ncu capture record, if it was taken on the
+    current kernel source; else None."""
     try:
-        txt = open(PROFILE_FILE).read()
-    except OSError:
+        with open(PROFILE_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
         return None
-    vals = {}
-    for line in txt.splitlines():
-        if ":" in line and line.strip().startswith("- "):
-            k, v = line.strip()[2:].split(":", 1)
-            vals[k.strip()] = v.strip().strip("`")
-    if vals.get("kernel_source_sha") != kernel_source_hash():
+    if rec.get("kernel_source_sha") != kernel_source_hash():
         return None
     try:
-        return float(vals["dram_bytes_per_full_launch"])
-    except (KeyError, ValueError):
+        return float(rec["dram_bytes_per_launch"])
+    except (KeyError, TypeError, ValueError):
         return None
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """SM clock, power and clock-event reasons of the benchmark's GPU, sampled
+    every 10 ms through NVML (read-only queries) while the timed region runs;
+    falls back to `nvidia-smi -lms 200`. summary() keeps the samples taken
+    between mark_start() and mark_stop() (host time around the region)."""
 
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    # NVML clocks-event reason bits
+    BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+            "sw_power_cap": 0x4}
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.rows = []
+    def __init__(self, cuda_index: int):
+        self.cuda_index = cuda_index
+        self.rows = []  # (host time, sm MHz, max MHz, power W, set of reasons)
         self.proc = None
         self.thread = None
+        self.stop_flag = threading.Event()
+        self.t0 = None
+        self.t1 = None
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.cuda_index)
+        uuid = getattr(props, "uuid", None)
+        if uuid is not None:
+            u = str(uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(u if u.startswith("GPU-") else "GPU-" + u)
+        bus = getattr(props, "pci_bus_id", None)
+        if bus is not None:
+            busid = (f"{getattr(props, 'pci_domain_id', 0):08X}:{bus:02X}:"
+                     f"{getattr(props, 'pci_device_id', 0):02X}.0")
+            return pynvml.nvmlDeviceGetHandleByPciBusId(busid)
+        return pynvml.nvmlDeviceGetHandleByIndex(self.cuda_index)
 
     def start(self):
         try:
+            import pynvml
+            h = self._nvml_handle()
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+
+            def loop():
+                while not self.stop_flag.is_set():
+                    try:
+                        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                        pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        bits = get_reasons(h)
+                        rs = {n for n, b in self.BITS.items() if bits & b}
+                        self.rows.append((time.perf_counter(), float(sm), float(mx), pw, rs))
+                    except Exception:  # noqa: BLE001 - a failed sample is skipped
+                        pass
+                    self.stop_flag.wait(0.01)
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            self.source = "nvml 10 ms"
+            return
+        except Exception:  # noqa: BLE001 - no NVML: fall back to nvidia-smi
+            pass
+        try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", "-i", str(self.cuda_index), f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "200"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
             return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.source = "nvidia-smi 200 ms"
+        self.thread = threading.Thread(target=self._read_smi, daemon=True)
         self.thread.start()
 
-    def _read(self):
+    def _read_smi(self):
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
         for line in self.proc.stdout:
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) >= 9:
-                self.rows.append(parts)
+            if len(parts) >= 9 and num(parts[1]) is not None:
+                rs = {self.NAMES[i] for i in range(4) if parts[5 + i].lower() == "active"}
+                self.rows.append((time.perf_counter(), num(parts[1]), num(parts[2]),
+                                  num(parts[3]), rs))
+
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_stop(self):
+        self.t1 = time.perf_counter()
 
     def stop(self):
+        self.stop_flag.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -127,23 +196,22 @@ class ClockSampler:
             self.thread.join(timeout=5)
 
     def summary(self):
-        if not self.rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        def num(x):
-            try:
-                return float(x)
-            except ValueError:
-                return None
-        sm = [num(r[1]) for r in self.rows if num(r[1]) is not None]
-        mx = [num(r[2]) for r in self.rows if num(r[2]) is not None]
-        pw = [num(r[3]) for r in self.rows if num(r[3]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in self.rows for i in range(4)
-                          if r[5 + i].lower() == "active"})
+        rows = self.rows
+        if self.t0 is not None and self.t1 is not None:
+            inside = [r for r in rows if self.t0 <= r[0] <= self.t1]
+            if inside:
+                rows = inside
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0,
+                    "source": self.source}
+        sm = [r[1] for r in rows if r[1] is not None]
+        mx = [r[2] for r in rows if r[2] is not None]
+        pw = [r[3] for r in rows if r[3] is not None]
+        reasons = sorted(set().union(*[r[4] for r in rows]))
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
                 "power_w": statistics.median(pw) if pw else None,
-                "samples": len(self.rows)}
+                "samples": len(rows), "source": self.source}
 
 
 def _dist():
@@ -333,7 +401,8 @@ def run_gpu(args, world, rank, local):
         dist.barrier()
     torch.cuda.synchronize()
     sampler.start()
-    time.sleep(0.3)  # let the sampler start before the timed region
+    time.sleep(0.1)  # let the sampler start before the timed region
+    sampler.mark_start()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     if args.flush_l2:
@@ -356,6 +425,7 @@ def run_gpu(args, world, rank, local):
         va.set_profile_events()
         t1.record(stream)
     torch.cuda.synchronize()
+    sampler.mark_stop()
     sampler.stop()
     if world > 1:
         dist.barrier()
@@ -431,6 +501,12 @@ def run_gpu(args, world, rank, local):
                   "peak_source": f"{peak_src} bf16_tflops (burst)",
                   "frac_of_sustained": achieved / float(peaks["bf16_tflops_sustained"])}
         rl["frac"] = rl["achieved"] / rl["peak"]
+        clk = sampler.summary()
+        rl["sm_mhz_median"] = clk["sm_mhz"]
+        if bound == "tensor":
+            rl["datasheet_peak"] = DATASHEET_BF16_TFLOPS
+            rl["frac_of_datasheet"] = achieved / DATASHEET_BF16_TFLOPS
+            rl["datasheet_source"] = DATASHEET_SOURCE
         rl["traffic"] = traffic
         rl["kernel"] = (f"attn_fwd_sm100<{w.head_dim},{str(w.bias_key is not None).lower()},"
                         f"{str(w.bias_pair is not None).lower()}>")
@@ -448,7 +524,7 @@ def run_gpu(args, world, rank, local):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms, "steps": e_steps},
             "gpu_launches": va.launches_per_call() * args.steps,
-            "clocks": sampler.summary(),
+            "clocks": clk,
         }
         if not args.no_cpu_baseline:
             r = oracle_sample_rate(w, budget_s=args.cpu_budget)
@@ -622,6 +698,8 @@ def run_backward(args, world, rank, local):
     torch.cuda.synchronize()
     clocks = ClockSampler(local)
     clocks.start()
+    time.sleep(0.1)
+    clocks.mark_start()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record()
@@ -629,6 +707,7 @@ def run_backward(args, world, rank, local):
         step()
     t1.record()
     torch.cuda.synchronize()
+    clocks.mark_stop()
     clocks.stop()
     clk = clocks.summary()
     ms = t0.elapsed_time(t1) / args.steps

@@ -370,6 +370,34 @@ int varlen_attn_get_device_error(void* stream);
  */
 int varlen_attn_set_profile_events(void* start_event, void* stop_event);
 
+/*
+ * Failure-detection control. Every wait of the tensor-core forward and
+ * backward kernels on a pipeline barrier (shared-memory mbarrier) is bounded:
+ * after `cycles` SM clock cycles without progress the kernel raises
+ * VARLEN_ATTN_ERR_DEVICE_TIMEOUT in the device error word, every role of the
+ * CTA leaves its loop, the copies already in flight are waited for (with a
+ * fixed limit of 2^29 cycles), tensor memory is released and the kernel
+ * returns; the outputs of that call are then undefined but the context stays
+ * usable. 0 restores the default of 2^33 cycles (about 4 s at 2 GHz).
+ * Applies to calls launched after it, from any host thread (process-wide).
+ * A short limit is a test of the abort path, not a tuning knob: any wait
+ * longer than the limit aborts the call. Negative values return
+ * VARLEN_ATTN_ERR_BAD_SHAPE. (No counterpart on the pages: their kernels have
+ * no failure detection.)
+ */
+int varlen_attn_set_wait_limit(long long cycles);
+
+/*
+ * Test hook of that abort path, off by default: while `on` is non-zero, the
+ * MMA warp of every CTA of the tensor-core forward and backward kernels
+ * launched afterwards first waits on a barrier phase that nothing completes,
+ * so that wait runs out after the wait limit and aborts the call exactly as
+ * a stalled pipeline would (VARLEN_ATTN_ERR_DEVICE_TIMEOUT, outputs
+ * undefined). Process-wide; pass 0 to switch it off. Use it together with a
+ * short varlen_attn_set_wait_limit, or each call waits the default ~4 s.
+ */
+int varlen_attn_set_test_stall(int on);
+
 /* Number of kernels one varlen_attn_fwd / varlen_attn_fwd_f32 call launches. */
 int varlen_attn_launches_per_call(int fp32_path);
 

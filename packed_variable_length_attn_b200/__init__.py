@@ -34,7 +34,8 @@ from typing import Optional, Sequence, Tuple
 __all__ = ["varlen_attn_fwd", "varlen_attn_fwd_noalloc", "library_path", "load_library", "VarlenAttnError",
            "get_device_error", "set_profile_events", "launches_per_call", "exported_symbols",
            "mask_to_seqlens", "gather_rows", "scatter_rows", "unpad", "pad", "fold_pair_bias_row",
-           "varlen_attn_decode", "varlen_attn_bwd", "BIAS_PAIR_KV_HEADS"]
+           "varlen_attn_decode", "varlen_attn_bwd", "set_wait_limit", "set_test_stall",
+           "BIAS_PAIR_KV_HEADS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libvarlen_attn.so")
@@ -63,7 +64,8 @@ def exported_symbols() -> Tuple[str, ...]:
             "varlen_attn_launches_per_call", "varlen_attn_version",
             "varlen_attn_last_error_detail", "varlen_attn_fwd_noalloc", "varlen_attn_fwd_ex",
             "varlen_mask_to_seqlens", "varlen_gather_rows", "varlen_scatter_rows",
-            "varlen_fold_pair_bias_row", "varlen_attn_decode", "varlen_attn_bwd")
+            "varlen_fold_pair_bias_row", "varlen_attn_decode", "varlen_attn_bwd",
+            "varlen_attn_set_wait_limit", "varlen_attn_set_test_stall")
 
 
 def load_library():
@@ -108,6 +110,10 @@ def load_library():
     lib.varlen_attn_get_device_error.restype = i32
     lib.varlen_attn_set_profile_events.argtypes = [vp, vp]
     lib.varlen_attn_set_profile_events.restype = i32
+    lib.varlen_attn_set_wait_limit.argtypes = [ctypes.c_longlong]
+    lib.varlen_attn_set_wait_limit.restype = i32
+    lib.varlen_attn_set_test_stall.argtypes = [i32]
+    lib.varlen_attn_set_test_stall.restype = i32
     lib.varlen_attn_launches_per_call.argtypes = [i32]
     lib.varlen_attn_launches_per_call.restype = i32
     lib.varlen_attn_version.argtypes = []
@@ -153,6 +159,21 @@ def set_profile_events(start=None, stop=None):
             raise ValueError("record the events once first (torch creates them lazily)")
         _check(lib.varlen_attn_set_profile_events(ctypes.c_void_p(start.cuda_event),
                                                   ctypes.c_void_p(stop.cuda_event)))
+
+
+def set_wait_limit(cycles: int = 0):
+    """Limit, in SM clock cycles, of every bounded barrier wait of the
+    tensor-core kernels launched afterwards (process-wide); 0 restores the
+    default (2^33). A wait that runs out raises status 10 in the device error
+    word and the call's outputs are undefined."""
+    _check(load_library().varlen_attn_set_wait_limit(int(cycles)))
+
+
+def set_test_stall(on: bool = False):
+    """Test hook of the abort path: while on, every tensor-core forward and
+    backward launch first waits on a barrier phase that nothing completes, so
+    the call ends with status 10 after the wait limit. Off by default."""
+    _check(load_library().varlen_attn_set_test_stall(1 if on else 0))
 
 
 def launches_per_call(fp32: bool = False) -> int:

@@ -57,6 +57,9 @@ constexpr float kLn2 = 0.6931471805599453f;
 // A row's running max is only moved (and O rescaled) when the tile max
 // exceeds it by more than this many powers of two; P stays <= 2^8.
 constexpr float kRescaleThreshold = 8.0f;
+// Default limit of a bounded wait (the launch parameter wait_limit; a caller
+// may shorten it to exercise the abort path) and the fixed limit of the
+// drains that follow an abort.
 constexpr long long kWaitLimitCycles = 1ll << 33;    // ~4 s at 2 GHz
 constexpr long long kDrainLimitCycles = 1ll << 29;   // ~0.3 s
 
@@ -91,6 +94,7 @@ struct KCfg {
 struct Ctl {
   volatile int* abort;
   int* error;
+  long long limit;  // cycles a wait may take before it raises kErrTimeout
 };
 
 __device__ __forceinline__ void raise_abort(const Ctl& c) {
@@ -105,7 +109,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const C
   while (true) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     if (*c.abort) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > c.limit) {
       raise_abort(c);
       return false;
     }
@@ -325,7 +329,7 @@ __device__ __forceinline__ void issue_pv_half(uint32_t o_tmem, uint32_t p_tmem, 
 // lane issues the tensor-core instructions and their commits. The slot loops
 // are unrolled so that every per-slot counter stays in a register.
 template <int D>
-__device__ void mma_role(const Smem<D>& sm, uint32_t tmem, const Ctl& ctl) {
+__device__ void mma_role(const Smem<D>& sm, uint32_t tmem, const Ctl& ctl, int test_stall) {
   using C = KCfg<D>;
   const unsigned FULL = 0xffffffffu;
   uint32_t kv_t = 0, q_uses[2] = {0, 0}, o_uses[2] = {0, 0};
@@ -344,7 +348,9 @@ __device__ void mma_role(const Smem<D>& sm, uint32_t tmem, const Ctl& ctl) {
     ++kv_t;
     return r;
   };
-  bool ok = true;
+  // Test hook: drain's phase 0 completes only through this warp's final
+  // commit, so this wait can only run out (and abort the CTA).
+  bool ok = !test_stall || wait(sm.drain(), 0);
   for (int it = 0; ok; ++it) {
     const int k = it & 1;
     if (!wait(sm.item_full(k), (it >> 1) & 1)) break;
@@ -802,7 +808,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *sm.tmem_slot();
-  const Ctl ctl{sm.abort_flag(), p.error};
+  const Ctl ctl{sm.abort_flag(), p.error, p.wait_limit};
 
   if (warp < 8) {
     ptx::setmaxnreg_inc<kSoftmaxRegs>();
@@ -810,7 +816,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else {
     ptx::setmaxnreg_dec<kWorkerRegs>();
     if (warp == kMmaWarp) {
-      mma_role<D>(sm, tmem, ctl);
+      mma_role<D>(sm, tmem, ctl, p.test_stall);
     } else if (warp == kLoadWarp) {
       load_role<D>(sm, &tm_q, &tm_k, &tm_v, p, ctl);
     }

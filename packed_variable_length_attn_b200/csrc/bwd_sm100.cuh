@@ -60,6 +60,9 @@ struct BwdParams {
   void* dk;                       // bf16 [Tk, Hkv, D]
   void* dv;                       // bf16 [Tk, Hkv, D]
   int* error;
+  long long wait_limit;           // cycles a bounded wait may take
+  int test_stall;                 // test hook: the MMA warp first waits on a barrier
+                                  // phase nothing completes (its wait runs out)
 };
 
 // Compute warps 0-15: warp w reads tensor-memory lanes 32(w % 4) .. +31 and
@@ -325,7 +328,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   BwdSmem<D> sm;
   const uint32_t tmem = bwd_setup<D>(sm, smem_raw);
-  const Ctl ctl{sm.abort_flag(), p.error};
+  const Ctl ctl{sm.abort_flag(), p.error, p.wait_limit};
   const int warp = threadIdx.x >> 5;
 
   if (warp == kBwdLoadWarp) {
@@ -349,7 +352,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint64_t kd = desc_kmajor_sw128(ptx::smem_u32(sm.fixed(0)));
     const uint64_t vd = desc_kmajor_sw128(ptx::smem_u32(sm.fixed(1)));
     using C = BwdCfg<D>;
-    bool ok = __all_sync(FULL, wait_bar(sm.fixed_full(), 0, ctl));
+    // Test hook: o_full's phase 0 completes only through this warp's final
+    // commit, so this wait can only run out (and abort the CTA).
+    bool ok = !p.test_stall || __all_sync(FULL, wait_bar(sm.o_full(), 0, ctl));
+    ok = ok && __all_sync(FULL, wait_bar(sm.fixed_full(), 0, ctl));
     auto a_addr = [&](int t) { return ptx::smem_u32(sm.ring_a(ring_stage<C::kNA>(t))); };
     auto b_addr = [&](int t) { return ptx::smem_u32(sm.ring_b(ring_stage<C::kNB>(t))); };
     auto issue_sT = [&](int t) {  // S^T(t) = K Q(t)^T
@@ -572,7 +578,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   BwdSmem<D> sm;
   const uint32_t tmem = bwd_setup<D>(sm, smem_raw);
-  const Ctl ctl{sm.abort_flag(), p.error};
+  const Ctl ctl{sm.abort_flag(), p.error, p.wait_limit};
   const int warp = threadIdx.x >> 5;
 
   if (warp == kBwdLoadWarp) {
@@ -597,7 +603,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint64_t qd = desc_kmajor_sw128(ptx::smem_u32(sm.fixed(0)));
     const uint64_t dod = desc_kmajor_sw128(ptx::smem_u32(sm.fixed(1)));
     using C = BwdCfg<D>;
-    bool ok = n_k == 0 || __all_sync(FULL, wait_bar(sm.fixed_full(), 0, ctl));
+    // Test hook: o_full's phase 0 completes only through this warp's final
+    // commit, so this wait can only run out (and abort the CTA).
+    bool ok = !p.test_stall || __all_sync(FULL, wait_bar(sm.o_full(), 0, ctl));
+    ok = ok && (n_k == 0 || __all_sync(FULL, wait_bar(sm.fixed_full(), 0, ctl)));
     auto a_addr = [&](int j) { return ptx::smem_u32(sm.ring_a(ring_stage<C::kNA>(j))); };
     auto b_addr = [&](int j) { return ptx::smem_u32(sm.ring_b(ring_stage<C::kNB>(j))); };
     auto issue_s_j = [&](int j) {  // S(j) = Q K(j)^T

@@ -58,6 +58,9 @@ struct AttnParams {
   float* lse;                      // [Hq, Tq] or null
   Workspace ws;
   int* error;
+  long long wait_limit;            // cycles a bounded wait may take
+  int test_stall;                  // test hook: the MMA warp first waits on a barrier
+                                   // phase nothing completes (its wait runs out)
 };
 
 // One CTA work item: up to two 128-row query tiles (slots) that stream the

@@ -10,6 +10,7 @@
 #include <cstring>
 #include <map>
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <utility>
 
@@ -66,6 +67,15 @@ thread_local char t_detail[256] = "";
 int cuda_fail(const char* step, cudaError_t e) {
   snprintf(t_detail, sizeof t_detail, "%s: %s (%d)", step, cudaGetErrorString(e), (int)e);
   return VARLEN_ATTN_ERR_CUDA;
+}
+
+// Limit of the kernels' bounded waits, in SM clock cycles (0 = default).
+std::atomic<long long> g_wait_limit{0};
+// Test hook of the abort path (varlen_attn_set_test_stall).
+std::atomic<int> g_test_stall{0};
+long long wait_limit() {
+  const long long v = g_wait_limit.load(std::memory_order_relaxed);
+  return v > 0 ? v : kWaitLimitCycles;
 }
 
 thread_local cudaEvent_t t_ev_start = nullptr;
@@ -219,7 +229,7 @@ int launch_schedule(const SchedParams& sp, cudaStream_t st) {
   static thread_local int configured_for = -1;
   int dev = 0;
   cudaGetDevice(&dev);
-  const int smem = kSortCap * (int)sizeof(unsigned long long);
+  const int smem = kSchedSmemBytes;
   if (configured_for != dev) {
     if (int rc = set_smem(schedule_kernel, smem)) return rc;
     configured_for = dev;
@@ -269,7 +279,7 @@ int fwd_bf16(const void* q, const void* k, const void* v, const int32_t* cu_seql
              int max_seqlen_k, int n_heads, int n_kv_heads, int head_dim, float softmax_scale,
              int causal, const float* bias_per_key, const float* bias_pair, int64_t bias_stride_b,
              int64_t bias_stride_h, int64_t bias_stride_q, int64_t bias_stride_k, unsigned flags,
-             void* out, float* lse, void* stream) {
+             void* out, float* lse, void* stream, bool fixed_scratch) {
   if (flags & ~(unsigned)VARLEN_ATTN_BIAS_PAIR_KV_HEADS) return VARLEN_ATTN_ERR_BAD_BIAS;
   Common a{batch, total_q, total_k, max_seqlen_q, max_seqlen_k, n_heads, n_kv_heads, head_dim,
            causal ? 1 : 0, cu_seqlens_q, cu_seqlens_k, bias_per_key, bias_pair, bias_stride_b,
@@ -289,8 +299,22 @@ int fwd_bf16(const void* q, const void* k, const void* v, const int32_t* cu_seql
   const int64_t capacity = (int64_t)batch * groups_per_seq;
   if (capacity * n_hg > INT32_MAX || capacity > (INT32_MAX / 16)) return VARLEN_ATTN_ERR_TOO_LARGE;
 
+  // The work list lives in the grow-only workspace, or, for the no-allocation
+  // entry point, in the fixed module array (never allocated, never cleared:
+  // the schedule kernel rewrites the counter, the count and every list entry
+  // it publishes before the attention kernel reads them).
   void* wsp = nullptr;
-  if ((rc = workspace(stream, 256 + 2 * (size_t)capacity * sizeof(int2), &wsp))) return rc;
+  if (fixed_scratch) {
+    if (capacity > kNoAllocMaxPairs) {
+      snprintf(t_detail, sizeof t_detail,
+               "work list of %lld (sequence, q-block group) pairs exceeds the fixed scratch of %d",
+               (long long)capacity, kNoAllocMaxPairs);
+      return VARLEN_ATTN_ERR_SCRATCH_LIMIT;
+    }
+    if ((rc = noalloc_scratch(&wsp))) return rc;
+  } else if ((rc = workspace(stream, 256 + 2 * (size_t)capacity * sizeof(int2), &wsp))) {
+    return rc;
+  }
   Workspace ws = carve(wsp, (int)capacity);
 
   CUtensorMap tq, tk, tv;
@@ -340,6 +364,8 @@ int fwd_bf16(const void* q, const void* k, const void* v, const int32_t* cu_seql
   prm.lse = lse;
   prm.ws = ws;
   prm.error = di->error_word;
+  prm.wait_limit = wait_limit();
+  prm.test_stall = g_test_stall.load(std::memory_order_relaxed);
 
   int64_t items = capacity * n_hg;
   const int grid = (int)(items < di->sm_count ? items : di->sm_count);
@@ -426,7 +452,7 @@ int varlen_attn_fwd(const void* q, const void* k, const void* v, const int32_t* 
   return fwd_bf16(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
                   max_seqlen_k, n_heads, n_kv_heads, head_dim, softmax_scale, causal, bias_per_key,
                   bias_pair, bias_stride_b, bias_stride_h, bias_stride_q, bias_stride_k, 0u, out,
-                  lse, stream);
+                  lse, stream, /*fixed_scratch=*/false);
 }
 
 int varlen_attn_fwd_ex(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
@@ -439,7 +465,7 @@ int varlen_attn_fwd_ex(const void* q, const void* k, const void* v, const int32_
   return fwd_bf16(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
                   max_seqlen_k, n_heads, n_kv_heads, head_dim, softmax_scale, causal, bias_per_key,
                   bias_pair, bias_stride_b, bias_stride_h, bias_stride_q, bias_stride_k, flags, out,
-                  lse, stream);
+                  lse, stream, /*fixed_scratch=*/false);
 }
 
 int varlen_attn_fwd_f32(const float* q, const float* k, const float* v,
@@ -536,99 +562,10 @@ int varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                             int causal, const float* bias_per_key, const float* bias_pair,
                             int64_t bias_stride_b, int64_t bias_stride_h, int64_t bias_stride_q,
                             int64_t bias_stride_k, void* out, float* lse, void* stream) {
-  Common a{batch, total_q, total_k, max_seqlen_q, max_seqlen_k, n_heads, n_kv_heads, head_dim,
-           causal ? 1 : 0, cu_seqlens_q, cu_seqlens_k, bias_per_key, bias_pair, bias_stride_b,
-           bias_stride_h, bias_stride_q, bias_stride_k};
-  int rc = validate_common(a, q, k, v, out, lse);
-  if (rc) return rc;
-  DeviceInfo* di = nullptr;
-  if ((rc = device_info(&di))) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (total_q == 0 || max_seqlen_q == 0) return VARLEN_ATTN_OK;
-
-  const int G = n_heads / n_kv_heads;
-  const int pairing = G >= 2 ? kPairHeads : kPairQBlocks;
-  const int n_hp = (G + 1) / 2;
-  const int n_hg = pairing == kPairHeads ? n_kv_heads * n_hp : n_heads;
-  const int64_t capacity = (int64_t)batch * seq_groups(max_seqlen_q, pairing);
-  if (capacity > kNoAllocMaxPairs) {
-    snprintf(t_detail, sizeof t_detail,
-             "work list of %lld (sequence, q-block group) pairs exceeds the fixed scratch of %d",
-             (long long)capacity, kNoAllocMaxPairs);
-    return VARLEN_ATTN_ERR_SCRATCH_LIMIT;
-  }
-  if (capacity * n_hg > INT32_MAX) return VARLEN_ATTN_ERR_TOO_LARGE;
-
-  void* wsp = nullptr;
-  if ((rc = noalloc_scratch(&wsp))) return rc;
-  // The schedule kernel rewrites the counter, the count and every list entry
-  // it publishes before the attention kernel reads them, so no clearing of
-  // the previous call's contents is needed.
-  Workspace ws = carve(wsp, (int)capacity);
-
-  CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, head_dim, n_heads, total_q, BM) ||
-      !make_tmap(&tk, k, head_dim, n_kv_heads, total_k, BN) ||
-      !make_tmap(&tv, v, head_dim, n_kv_heads, total_k, BN))
-    return VARLEN_ATTN_ERR_CUDA;
-
-  SchedParams sp;
-  sp.cu_q = cu_seqlens_q;
-  sp.cu_k = cu_seqlens_k;
-  sp.batch = batch;
-  sp.total_q = total_q;
-  sp.total_k = total_k;
-  sp.max_q = max_seqlen_q;
-  sp.max_k = max_seqlen_k;
-  sp.causal = a.causal;
-  sp.pairing = pairing;
-  sp.n_hg = n_hg;
-  sp.ws = ws;
-  sp.error = di->error_word;
-  if ((rc = launch_schedule(sp, st))) return rc;
-
-  AttnParams prm;
-  prm.cu_q = cu_seqlens_q;
-  prm.cu_k = cu_seqlens_k;
-  prm.total_q = total_q;
-  prm.n_heads = n_heads;
-  prm.n_kv_heads = n_kv_heads;
-  prm.group = G;
-  prm.pairing = pairing;
-  prm.n_hp = n_hp;
-  prm.n_hg = n_hg;
-  prm.causal = a.causal;
-  prm.scale_log2 = softmax_scale * 1.4426950408889634f;
-  prm.scale = softmax_scale;
-  prm.bias_key = bias_per_key;
-  prm.bias_pair = bias_pair;
-  prm.sb = bias_stride_b;
-  prm.sh = bias_stride_h;
-  prm.bias_head_div = 1;
-  prm.sr = bias_stride_q;
-  prm.sc = bias_stride_k;
-  prm.pair_vec = bias_pair && bias_stride_k == 1 && aligned(bias_pair, 16) &&
-                 bias_stride_b % 4 == 0 && bias_stride_h % 4 == 0 && bias_stride_q % 4 == 0;
-  prm.out = out;
-  prm.lse = lse;
-  prm.ws = ws;
-  prm.error = di->error_word;
-
-  const int64_t items = capacity * n_hg;
-  const int grid = (int)(items < di->sm_count ? items : di->sm_count);
-  const bool bk = bias_per_key != nullptr, bp = bias_pair != nullptr;
-  if (head_dim == 64) {
-    if (bk && bp) rc = launch_attn<64, true, true>(grid, tq, tk, tv, prm, st);
-    else if (bk) rc = launch_attn<64, true, false>(grid, tq, tk, tv, prm, st);
-    else if (bp) rc = launch_attn<64, false, true>(grid, tq, tk, tv, prm, st);
-    else rc = launch_attn<64, false, false>(grid, tq, tk, tv, prm, st);
-  } else {
-    if (bk && bp) rc = launch_attn<128, true, true>(grid, tq, tk, tv, prm, st);
-    else if (bk) rc = launch_attn<128, true, false>(grid, tq, tk, tv, prm, st);
-    else if (bp) rc = launch_attn<128, false, true>(grid, tq, tk, tv, prm, st);
-    else rc = launch_attn<128, false, false>(grid, tq, tk, tv, prm, st);
-  }
-  return rc;
+  return fwd_bf16(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+                  max_seqlen_k, n_heads, n_kv_heads, head_dim, softmax_scale, causal, bias_per_key,
+                  bias_pair, bias_stride_b, bias_stride_h, bias_stride_q, bias_stride_k, 0u, out,
+                  lse, stream, /*fixed_scratch=*/true);
 }
 
 const char* varlen_attn_strerror(int status) {
@@ -952,6 +889,8 @@ int varlen_attn_bwd(const void* q, const void* k, const void* v, const void* out
   bp.dk = dk;
   bp.dv = dv;
   bp.error = di->error_word;
+  bp.wait_limit = wait_limit();
+  bp.test_stall = g_test_stall.load(std::memory_order_relaxed);
   const dim3 grid_a((unsigned)std::max(1, ceil_div(max_seqlen_k, BN)), (unsigned)n_kv_heads,
                     (unsigned)batch);
   const dim3 grid_q((unsigned)std::max(1, ceil_div(max_seqlen_q, BM)), (unsigned)n_heads,
@@ -969,6 +908,17 @@ int varlen_attn_bwd(const void* q, const void* k, const void* v, const void* out
     else rc = launch_bwd<128, false, false>(grid_a, grid_q, tq, tk, tv, tdo, bp, st);
   }
   return rc;
+}
+
+int varlen_attn_set_wait_limit(long long cycles) {
+  if (cycles < 0) return VARLEN_ATTN_ERR_BAD_SHAPE;
+  g_wait_limit.store(cycles, std::memory_order_relaxed);
+  return VARLEN_ATTN_OK;
+}
+
+int varlen_attn_set_test_stall(int on) {
+  g_test_stall.store(on ? 1 : 0, std::memory_order_relaxed);
+  return VARLEN_ATTN_OK;
 }
 
 int varlen_attn_launches_per_call(int fp32_path) {

@@ -88,8 +88,28 @@ def sample_rows(w, n, seed):
     return [x[0] for x in s], [x[1] for x in s], [x[2] for x in s]
 
 
-def compare_sampled(w, out, lse, n=256, seed=0):
-    seq, head, row = sample_rows(w, n, seed)
+def stratified_rows(w, rows_per_block=4, seed=0):
+    """(seq, head, local row) samples covering every (sequence, 128-row
+    q-block): its first and last row plus rows_per_block - 2 random rows,
+    each on one head drawn at random from every K/V group."""
+    g = np.random.default_rng(seed)
+    G = w.n_heads // w.n_kv_heads
+    out = set()
+    for i in range(w.batch):
+        L = w.lengths_q[i]
+        for b0 in range(0, L, 128):
+            b1 = min(b0 + 128, L) - 1
+            rows = {b0, b1}
+            while len(rows) < min(rows_per_block, b1 - b0 + 1):
+                rows.add(int(g.integers(b0, b1 + 1)))
+            for r in rows:
+                for kvh in range(w.n_kv_heads):
+                    out.add((i, kvh * G + int(g.integers(G)), r))
+    s = sorted(out)
+    return [x[0] for x in s], [x[1] for x in s], [x[2] for x in s]
+
+
+def compare_rows(w, out, lse, seq, head, row):
     ro, rl = oracle.rows(w.q, w.k, w.v, w.cu_q, w.cu_k, w.n_heads, w.n_kv_heads,
                          w.softmax_scale, w.causal, seq, head, row, bias_key=w.bias_key,
                          bias_pair=w.bias_pair, bias_strides=w.bias_strides)
@@ -98,3 +118,11 @@ def compare_sampled(w, out, lse, n=256, seed=0):
     go = out.cpu()[t, h]
     gl = lse.cpu()[h, t]
     return compare(go, gl, ro, rl)
+
+
+def compare_sampled(w, out, lse, n=256, seed=0):
+    return compare_rows(w, out, lse, *sample_rows(w, n, seed))
+
+
+def compare_stratified(w, out, lse, rows_per_block=4, seed=0):
+    return compare_rows(w, out, lse, *stratified_rows(w, rows_per_block, seed))

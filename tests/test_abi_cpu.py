@@ -179,3 +179,19 @@ def test_backward_binding_rejects_bad_tensors(lib):
     # dout of the wrong shape
     with pytest.raises(ValueError):
         va.varlen_attn_bwd(q, k, k, q, lse, q[:2], cu, cu, 4, 4)
+
+
+def test_wait_limit_setting(lib):
+    # host-only: a negative limit is rejected, 0 restores the default
+    assert lib.varlen_attn_set_wait_limit(-1) == 2
+    assert lib.varlen_attn_set_wait_limit(1000) == 0
+    assert lib.varlen_attn_set_wait_limit(0) == 0
+    with pytest.raises(va.VarlenAttnError):
+        va.set_wait_limit(-5)
+    va.set_wait_limit(0)
+
+
+def test_test_stall_setting(lib):
+    assert lib.varlen_attn_set_test_stall(1) == 0
+    assert lib.varlen_attn_set_test_stall(0) == 0
+    va.set_test_stall(False)

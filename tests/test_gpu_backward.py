@@ -27,7 +27,7 @@ MAX_ABS_FRAC = 2e-2
 @pytest.fixture(scope="module", autouse=True)
 def _cuda():
     if not torch.cuda.is_available():
-        pytest.skip("needs a CUDA device")
+        pytest.fail("CUDA device required for -m gpu tests")
     va.get_device_error()
     yield
     assert va.get_device_error() == 0

@@ -14,7 +14,7 @@ pytestmark = pytest.mark.gpu
 @pytest.fixture(scope="module", autouse=True)
 def _cuda():
     if not torch.cuda.is_available():
-        pytest.skip("needs a CUDA device")
+        pytest.fail("CUDA device required for -m gpu tests")
     va.get_device_error()
     yield
     assert va.get_device_error() == 0

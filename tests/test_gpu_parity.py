@@ -1,10 +1,12 @@
 """GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
 
 Full element-by-element comparisons on inputs the oracle finishes in
-seconds (several 128-row tiles and ragged tails), sampled rows on the five
-named workloads at their full sizes in the launch configuration the
-benchmark times, edge cases, and the bit-exact invariants (row isolation,
-packed-vs-solo, sequence order, run-to-run determinism).
+seconds (several 128-row tiles and ragged tails) and on the tiny, GenRec,
+graph-batch and short-query workloads at their full sizes; a stratified
+sample of the long causal GQA workload (every sequence and q-block, every
+K/V group) at its full size in the launch configuration the benchmark times;
+edge cases; and the bit-exact invariants (row isolation, packed-vs-solo,
+sequence order, run-to-run determinism) on every named workload.
 """
 import zlib
 
@@ -15,7 +17,7 @@ import torch
 import oracle
 from packed_variable_length_attn_b200 import (VarlenAttnError, get_device_error,
                                               varlen_attn_fwd, workloads)
-from tests.parity import compare, compare_sampled, run_gpu, run_oracle, to_device
+from tests.parity import compare, compare_stratified, run_gpu, run_oracle, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -90,12 +92,42 @@ def test_pair_bias_per_head_and_permuted_view():
     compare(out2, lse2, *run_oracle(w))
 
 
-@pytest.mark.parametrize("config", [2, 3, 4, 5])
-def test_named_workloads_sampled(config):
+@pytest.mark.parametrize("config", [2, 3, 4])
+def test_named_workloads_full_parity(config):
+    """Every output element of the GenRec, graph-batch and short-query
+    workloads at their full sizes, in the benchmark's launch configuration."""
     w = workloads.make(config)
     out, lse = run_gpu(w)
-    res = compare_sampled(w, out, lse, n=192, seed=config)
+    res = compare(out, lse, *run_oracle(w))
     print(config, res)
+
+
+def test_long_workload_stratified_parity():
+    """The long causal GQA workload (the benchmark's) at full size: every
+    (sequence, 128-row q-block) is checked on its first and last row and two
+    random rows, each on one head drawn from every K/V group."""
+    w = workloads.make(5)
+    out, lse = run_gpu(w)
+    res = compare_stratified(w, out, lse, rows_per_block=4, seed=5)
+    print(res)
+
+
+@pytest.mark.parametrize("batch,causal,hq,hkv", [(16385, True, 2, 1), (40000, False, 2, 2),
+                                                  (40000, True, 4, 2)])
+def test_packs_beyond_one_shared_memory_sort(batch, causal, hq, hkv):
+    """More sequences than the schedule sorts in one shared-memory pass: its
+    runs are merged in global memory. Every row must still be computed
+    exactly once (outputs start as NaN)."""
+    g = np.random.default_rng(batch + hq)
+    lq = [int(x) for x in g.integers(0, 41, batch)]
+    lq[batch // 2] = 300  # one longer sequence (several q-blocks)
+    w = workloads.make_custom(lq, None, n_heads=hq, n_kv_heads=hkv, head_dim=64, causal=causal,
+                              seed=batch)
+    dev = to_device(w)
+    out = torch.full_like(dev["q"], float("nan"))
+    lse = torch.full((w.n_heads, w.total_q), float("nan"), device="cuda")
+    run_gpu(w, dev=dev, out=out, lse=lse)
+    compare(out, lse, *run_oracle(w))
 
 
 def test_fp32_path_parity():
@@ -117,7 +149,7 @@ def _bits(t):
     return t.contiguous().view(torch.int16 if t.dtype == torch.bfloat16 else torch.int32).cpu()
 
 
-@pytest.mark.parametrize("config", [1, 2, 3, 4])
+@pytest.mark.parametrize("config", [1, 2, 3, 4, 5])
 def test_row_isolation_bit_exact(config):
     """Rewrite sequence 0's Q/K/V (and biases): every other sequence's output
     and LSE stay bit-identical."""
@@ -139,7 +171,7 @@ def test_row_isolation_bit_exact(config):
     assert not torch.equal(_bits(out2[:lq0]), _bits(out1[:lq0]))
 
 
-@pytest.mark.parametrize("config", [1, 2, 3, 4])
+@pytest.mark.parametrize("config", [1, 2, 3, 4, 5])
 def test_packed_vs_solo_bit_exact(config):
     """Each sequence run alone (batch of one) gives bit-identical O and LSE
     to its slice of the packed run."""
@@ -164,23 +196,26 @@ def test_packed_vs_solo_bit_exact(config):
         assert torch.equal(_bits(l1), _bits(lse[:, qa:qb])), i
 
 
-def test_sequence_order_permutation_bit_exact():
-    w = workloads.make(2)
+@pytest.mark.parametrize("config", [2, 4, 5])
+def test_sequence_order_permutation_bit_exact(config):
+    """The pack in reverse order gives every sequence bit-identical O and LSE."""
+    w = workloads.make(config)
     out, lse = run_gpu(w)
     perm = list(reversed(range(w.batch)))
     lq = [w.lengths_q[i] for i in perm]
+    lk = [w.lengths_k[i] for i in perm]
     q = torch.cat([w.q[w.cu_q[i]:w.cu_q[i + 1]] for i in perm])
     k = torch.cat([w.k[w.cu_k[i]:w.cu_k[i + 1]] for i in perm])
     v = torch.cat([w.v[w.cu_k[i]:w.cu_k[i + 1]] for i in perm])
-    w2 = workloads.make_custom(lq, n_heads=w.n_heads, n_kv_heads=w.n_kv_heads,
-                               head_dim=w.head_dim, causal=True, seed=0)
+    w2 = workloads.make_custom(lq, lk, n_heads=w.n_heads, n_kv_heads=w.n_kv_heads,
+                               head_dim=w.head_dim, causal=w.causal, seed=0)
     w2.q, w2.k, w2.v = q, k, v
     out2, lse2 = run_gpu(w2)
     for j, i in enumerate(perm):
         a, b = int(w.cu_q[i]), int(w.cu_q[i + 1])
         a2, b2 = int(w2.cu_q[j]), int(w2.cu_q[j + 1])
-        assert torch.equal(_bits(out2[a2:b2]), _bits(out[a:b]))
-        assert torch.equal(_bits(lse2[:, a2:b2]), _bits(lse[:, a:b]))
+        assert torch.equal(_bits(out2[a2:b2]), _bits(out[a:b])), i
+        assert torch.equal(_bits(lse2[:, a2:b2]), _bits(lse[:, a:b])), i
 
 
 def test_run_to_run_deterministic():
