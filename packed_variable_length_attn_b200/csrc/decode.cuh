@@ -16,8 +16,10 @@
 // (packed like q, [total_q, n_kv_heads, D]) are first written into the cache
 // after the cached ones and are then attended to as well.
 #pragma once
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
+#include "attn_sm100.cuh"  // Ctl, bounded barrier waits
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -380,6 +382,275 @@ __global__ void __launch_bounds__(kDecThreads) decode_combine_kernel(DecodeParam
     for (int j = 0; j < D / 32; ++j) p.out[e * D + lane + 32 * j] = __float2bfloat16_rn(o[j] * inv);
     if (lane == 0 && p.lse)
       p.lse[(long long)h * p.total_q + t] = wsum > 0.f ? mx + __logf(wsum) : -INFINITY;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Decode with a TMA ring and warp-owned key blocks, for up to kDec2MaxRows
+// query rows per (sequence, K/V head) (q_len x G; a decode step with G <= 8).
+//
+// One CTA per (key split, K/V head, sequence), five warps:
+//   warp 4      producer: one lane issues the TMA tile loads of each 32-key
+//               block (K then V, 64-column 128-byte-swizzled boxes of the
+//               cache [batch * cache_len, n_kv_heads, D]) into a kDec2Stages
+//               mbarrier ring;
+//   warps 0-3   consumers: warp w takes blocks w, w + 4, ... of the split and
+//               keeps its own online softmax (max, sum, O) for every row:
+//               scores with one key per lane (the key's row is read once and
+//               used for every query row), the block's max and sum by warp
+//               shuffles, P V with four (head_dim 128) or two (64) output
+//               dims per lane and P broadcast from shared memory.
+// No CTA barrier runs inside the loop; at the end the four warps' states are
+// merged in a fixed order (deterministic), as several key splits are by the
+// combine kernel. Keys at or past the sequence's length are masked in the
+// scores and skipped in P V, so whatever the cache holds there (old rows,
+// NaN) never reaches the output. Every barrier wait is bounded (Ctl): on
+// expiry the error word gets kErrTimeout and the CTA returns.
+constexpr int kDec2Consumers = 4;
+constexpr int kDec2Threads = 32 * (kDec2Consumers + 1);
+constexpr int kDec2Stages = 4;
+constexpr int kDec2MaxRows = 8;
+
+template <int D, int RT>
+struct Dec2Cfg {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kBox = kDecKeys * 128;        // 32 rows x 128 B (64 dims)
+  static constexpr int kTile = kChunks * kBox;       // K (or V) of one block
+  static constexpr int kStage = 2 * kTile;           // K then V
+  static constexpr int kQOff = kDec2Stages * kStage;             // q [RT][D] fp32
+  static constexpr int kPOff = kQOff + RT * D * 4;               // P [warp][32][RT] fp32
+  static constexpr int kBarOff = kPOff + kDec2Consumers * kDecKeys * RT * 4;
+  static constexpr int kMiscOff = kBarOff + 2 * kDec2Stages * 8;  // abort flag
+  static constexpr int kBytes = kMiscOff + 16 + 1024;             // + alignment slack
+  // the merge at the end reuses the ring: per warp m, l [RT] and O [RT][D]
+  static_assert(kDec2Consumers * RT * (D + 2) * 4 <= kDec2Stages * kStage, "merge area");
+};
+
+template <int D, int RT>
+__global__ void __launch_bounds__(kDec2Threads) decode_tma_kernel(
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+    DecodeParams p, long long wait_limit) {
+  extern __shared__ uint8_t dsm_raw[];
+  using C = Dec2Cfg<D, RT>;
+  constexpr int kDPL = D / 32;  // output dims per lane in P V
+  uint8_t* sm;
+  {
+    const uint32_t a = ptx::smem_u32(dsm_raw);
+    sm = dsm_raw + ((1024 - (a & 1023)) & 1023);  // 128-byte swizzle: 1024-byte aligned
+  }
+  float* qs = reinterpret_cast<float*>(sm + C::kQOff);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + C::kBarOff);
+  uint64_t* empty = full + kDec2Stages;
+  int* abort_flag = reinterpret_cast<int*>(sm + C::kMiscOff);
+
+  const int split = blockIdx.x, g = blockIdx.y, i = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int q0 = p.cu_q[i], Lq = p.cu_q[i + 1] - q0;
+  const int G = p.group;
+  const int R = Lq * G;
+  if (Lq <= 0) return;
+  const int Lk = p.cache_seqlens[i] + (p.k_new ? Lq : 0);
+  if (R > RT || Lk > p.cache_len || Lk < 0) {
+    if (tid == 0) atomicCAS(p.error, 0, kErrBadSeqlens);
+    return;
+  }
+  const int nblk_all = (Lk + kDecKeys - 1) / kDecKeys;
+  const int per = (nblk_all + p.n_splits - 1) / p.n_splits;
+  const int b0 = split * per, b1 = min(nblk_all, b0 + per);
+  const int nblk = max(0, b1 - b0);
+
+  if (tid == 0) {
+    for (int st = 0; st < kDec2Stages; ++st) {
+      ptx::mbar_init(full + st, 1);
+      ptx::mbar_init(empty + st, 1);
+    }
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  for (int e = tid; e < RT * D; e += kDec2Threads) {
+    const int rho = e / D, d = e - rho * D;
+    float v = 0.f;
+    if (rho < R) {
+      const int r = rho / G, hl = rho - r * G;
+      v = __bfloat162float(p.q[((long long)(q0 + r) * p.n_heads + g * G + hl) * D + d]);
+    }
+    qs[e] = v;
+  }
+  __syncthreads();
+  const Ctl ctl{abort_flag, p.error, wait_limit};
+  const long long row0 = (long long)i * p.cache_len;  // first cache row of sequence i
+
+  float m[RT], l[RT];
+  float o[RT][kDPL];
+#pragma unroll
+  for (int r = 0; r < RT; ++r) {
+    m[r] = -INFINITY;
+    l[r] = 0.f;
+#pragma unroll
+    for (int d = 0; d < kDPL; ++d) o[r][d] = 0.f;
+  }
+
+  if (warp == kDec2Consumers) {
+    // ---- producer
+    int t = 0;
+    for (; t < nblk; ++t) {
+      const int st = t % kDec2Stages;
+      if (!__all_sync(0xffffffffu, wait_bar(empty + st, ((t / kDec2Stages) & 1) ^ 1, ctl))) break;
+      if (ptx::elect_one()) {
+        uint8_t* dst = sm + st * C::kStage;
+        const int row = (int)(row0 + (long long)(b0 + t) * kDecKeys);
+        ptx::mbar_arrive_expect_tx(full + st, C::kStage);
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c) {
+          ptx::tma_load_3d(dst + c * C::kBox, &tm_k, full + st, c * 64, g, row);
+          ptx::tma_load_3d(dst + C::kTile + c * C::kBox, &tm_v, full + st, c * 64, g, row);
+        }
+      }
+      __syncwarp();
+    }
+    // wait (bounded) for every copy issued into each stage
+    for (int st = 0; st < kDec2Stages && st < t; ++st) {
+      const int uses = (t - 1 - st) / kDec2Stages + 1;
+      drain_bar(full + st, (uses - 1) & 1);
+    }
+  } else {
+    // ---- consumer warp: blocks t = warp, warp + 4, ...
+    float* pw = reinterpret_cast<float*>(sm + C::kPOff) + warp * kDecKeys * RT;  // [32][RT]
+    const int q_last = Lk - Lq;  // bottom-right causal: row r sees keys <= r + q_last
+    for (int t = warp; t < nblk; t += kDec2Consumers) {
+      const int st = t % kDec2Stages;
+      if (!__all_sync(0xffffffffu, wait_bar(full + st, (t / kDec2Stages) & 1, ctl))) break;
+      const uint8_t* kt = sm + st * C::kStage;
+      const uint8_t* vt = kt + C::kTile;
+      const int k0 = (b0 + t) * kDecKeys;
+      const int key = k0 + lane;
+      // scores: this lane's key against every row (row `lane` of each box,
+      // 16-byte unit u stored at unit u ^ (lane & 7))
+      uint64_t acc[RT];
+#pragma unroll
+      for (int r = 0; r < RT; ++r) acc[r] = 0ull;
+#pragma unroll
+      for (int c = 0; c < C::kChunks; ++c) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 kv = ptx::ld_shared_v4(ptx::smem_u32(kt + c * C::kBox + lane * 128 +
+                                                           ((u ^ (lane & 7)) << 4)));
+          const uint64_t k01 = ptx::f2(bf16_lo(kv.x), bf16_hi(kv.x));
+          const uint64_t k23 = ptx::f2(bf16_lo(kv.y), bf16_hi(kv.y));
+          const uint64_t k45 = ptx::f2(bf16_lo(kv.z), bf16_hi(kv.z));
+          const uint64_t k67 = ptx::f2(bf16_lo(kv.w), bf16_hi(kv.w));
+          const int d0 = c * 64 + u * 8;
+#pragma unroll
+          for (int r = 0; r < RT; ++r) {
+            const ulonglong2 qa = *reinterpret_cast<const ulonglong2*>(qs + r * D + d0);
+            const ulonglong2 qb = *reinterpret_cast<const ulonglong2*>(qs + r * D + d0 + 4);
+            acc[r] = ptx::ffma2(qa.x, k01, acc[r]);
+            acc[r] = ptx::ffma2(qa.y, k23, acc[r]);
+            acc[r] = ptx::ffma2(qb.x, k45, acc[r]);
+            acc[r] = ptx::ffma2(qb.y, k67, acc[r]);
+          }
+        }
+      }
+      // online softmax per row (log2 domain); masked keys give P = 0 exactly
+#pragma unroll
+      for (int r = 0; r < RT; ++r) {
+        float lo, hi;
+        ptx::f2_split(acc[r], lo, hi);
+        const bool vis = r < R && key < Lk && (!p.causal || key <= r / G + q_last);
+        const float s = vis ? (lo + hi) * p.scale_log2 : -INFINITY;
+        float mx = s;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const float m_new = fmaxf(m[r], mx);
+        const float mb = m_new == -INFINITY ? 0.f : m_new;
+        const float pr = ptx::ex2(s - mb);
+        float sum = pr;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        const float fac = ptx::ex2(m[r] - mb);  // 0 while m[r] is -inf
+        l[r] = l[r] * fac + sum;
+        m[r] = m_new;
+#pragma unroll
+        for (int d = 0; d < kDPL; ++d) o[r][d] *= fac;
+        pw[lane * RT + r] = pr;
+      }
+      __syncwarp();
+      // P V: this lane's output dims d0 .. d0 + kDPL - 1 over the block's keys
+      const int d0 = lane * kDPL;
+      const int vc = d0 / 64, vb = (d0 % 64) * 2;  // chunk, byte offset in the 128-byte row
+      const int nk = min(kDecKeys, Lk - k0);       // keys past the length are skipped
+      for (int kk = 0; kk < nk; ++kk) {
+        const uint32_t va = ptx::smem_u32(vt + vc * C::kBox + kk * 128) +
+                            (uint32_t)(((((vb >> 4) ^ (kk & 7)) << 4)) | (vb & 15));
+        float v[kDPL];
+        if constexpr (kDPL == 4) {
+          uint32_t x, y;
+          asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(x), "=r"(y) : "r"(va));
+          v[0] = bf16_lo(x); v[1] = bf16_hi(x); v[2] = bf16_lo(y); v[3] = bf16_hi(y);
+        } else {
+          uint32_t x;
+          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(x) : "r"(va));
+          v[0] = bf16_lo(x); v[1] = bf16_hi(x);
+        }
+        const float* prow = pw + kk * RT;
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          const float pr = prow[r];
+#pragma unroll
+          for (int d = 0; d < kDPL; ++d) o[r][d] = fmaf(pr, v[d], o[r][d]);
+        }
+      }
+      __syncwarp();  // pw is rewritten by the next block
+      if (lane == 0) ptx::mbar_arrive(empty + st);
+    }
+  }
+  __syncthreads();  // every copy has landed and every block has been read
+
+  // merge the consumer warps' states (fixed order) in the ring's space
+  float* mm = reinterpret_cast<float*>(sm);                    // [warp][RT]
+  float* ll = mm + kDec2Consumers * RT;                        // [warp][RT]
+  float* oo = ll + kDec2Consumers * RT;                        // [warp][RT][D]
+  if (warp < kDec2Consumers) {
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+      if (lane == 0) {
+        mm[warp * RT + r] = m[r];
+        ll[warp * RT + r] = l[r];
+      }
+#pragma unroll
+      for (int d = 0; d < kDPL; ++d) oo[(warp * RT + r) * D + lane * kDPL + d] = o[r][d];
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < R * D; e += kDec2Threads) {
+    const int rho = e / D, d = e - rho * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kDec2Consumers; ++w) M = fmaxf(M, mm[w * RT + rho]);
+    const float mb = M == -INFINITY ? 0.f : M;
+    float L = 0.f, O = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDec2Consumers; ++w) {
+      const float f = ptx::ex2(mm[w * RT + rho] - mb);
+      L += ll[w * RT + rho] * f;
+      O += oo[(w * RT + rho) * D + d] * f;
+    }
+    const int r = rho / G, h = g * G + (rho - r * G);
+    const float val = L > 0.f ? O / L : 0.f;
+    const long long oi = ((long long)(q0 + r) * p.n_heads + h) * D + d;
+    if (p.n_splits == 1)
+      p.out[oi] = __float2bfloat16_rn(val);
+    else
+      p.part_o[(long long)split * p.total_q * p.n_heads * D + oi] = val;
+    if (d == 0) {
+      const float lse = L > 0.f ? (M + __log2f(L)) * 0.6931471805599453f : -INFINITY;
+      const long long li = (long long)h * p.total_q + q0 + r;
+      if (p.n_splits == 1) {
+        if (p.lse) p.lse[li] = lse;
+      } else {
+        p.part_lse[(long long)split * p.n_heads * p.total_q + li] = lse;
+      }
+    }
   }
 }
 

@@ -410,6 +410,15 @@ int rows_args_ok(const void* src, int64_t src_rows, int64_t row_bytes, const int
 }
 
 template <int D, int RT>
+int launch_decode_tma(dim3 grid, const CUtensorMap& tk, const CUtensorMap& tv,
+                      const DecodeParams& dp, cudaStream_t st) {
+  auto kern = decode_tma_kernel<D, RT>;
+  if (int rc = set_smem(kern, Dec2Cfg<D, RT>::kBytes)) return rc;
+  kern<<<grid, kDec2Threads, Dec2Cfg<D, RT>::kBytes, st>>>(tk, tv, dp, wait_limit());
+  return check_launch("launch decode_tma_kernel");
+}
+
+template <int D, int RT>
 int launch_decode(dim3 grid, const DecodeParams& dp, cudaStream_t st) {
   auto kern = decode_kernel<D, RT>;
   if (int rc = set_smem(kern, DecSmem<D, RT>::kBytes)) return rc;
@@ -743,7 +752,24 @@ int varlen_attn_decode(const void* q, const int32_t* cu_seqlens_q, int batch, in
   const int rows_needed = max_seqlen_q * G;
   const int RT = rows_needed <= 4 ? 4 : rows_needed <= 8 ? 8 : rows_needed <= 16 ? 16 : 32;
   int rc = VARLEN_ATTN_OK;
-  if (head_dim == 64) {
+  if (RT <= kDec2MaxRows) {
+    // up to 8 rows per K/V head: TMA ring, warp-owned key blocks
+    CUtensorMap tk, tv;
+    const int cache_rows = batch * cache_len;
+    if (!make_tmap(&tk, k_cache, head_dim, n_kv_heads, cache_rows, kDecKeys) ||
+        !make_tmap(&tv, v_cache, head_dim, n_kv_heads, cache_rows, kDecKeys))
+      return VARLEN_ATTN_ERR_CUDA;
+    if (head_dim == 64)
+      rc = RT == 4 ? launch_decode_tma<64, 4>(grid, tk, tv, dp, st)
+                   : launch_decode_tma<64, 8>(grid, tk, tv, dp, st);
+    else
+      rc = RT == 4 ? launch_decode_tma<128, 4>(grid, tk, tv, dp, st)
+                   : launch_decode_tma<128, 8>(grid, tk, tv, dp, st);
+    if (!rc && splits > 1) {
+      if (head_dim == 64) decode_combine_kernel<64><<<rows, kDecThreads, 0, st>>>(dp);
+      else decode_combine_kernel<128><<<rows, kDecThreads, 0, st>>>(dp);
+    }
+  } else if (head_dim == 64) {
     switch (RT) {
       case 4: rc = launch_decode<64, 4>(grid, dp, st); break;
       case 8: rc = launch_decode<64, 8>(grid, dp, st); break;

@@ -82,6 +82,31 @@ def test_decode_parity(case):
     compare(out, lse, ref_o, ref_l)
 
 
+@pytest.mark.parametrize("hq,hkv,d,lq", [(32, 8, 128, 1), (14, 2, 64, 1), (8, 2, 128, 8)])
+def test_decode_ignores_cache_rows_past_each_length(hq, hkv, d, lq):
+    """Cache rows at and past each sequence's length hold NaN: the output is
+    finite and equals the result over the valid rows (keys there are masked
+    in the scores and never multiplied in P V)."""
+    cache_lens = [0, 1, 31, 32, 33, 1000, 4095]
+    lqs = [lq] * len(cache_lens)
+    cu_q, q, kc, vc, cs, _, _ = _case(77 + d, lqs, cache_lens, 4096 + 8, hq, hkv, d, False)
+    kn = torch.zeros(1)  # unused
+    kcn, vcn = kc.clone(), vc.clone()
+    for i, L in enumerate(cache_lens):
+        kcn[i, L:] = float("nan")
+        vcn[i, L:] = float("nan")
+    scale = 1.0 / np.sqrt(d)
+    for splits in (0, 1, 3):
+        out, lse = va.varlen_attn_decode(q.cuda(), cu_q.cuda(), lq, kcn.cuda(), vcn.cuda(),
+                                         cs.cuda(), softmax_scale=scale, causal=True,
+                                         num_splits=splits)
+        torch.cuda.synchronize()
+        assert torch.isfinite(out.float()).all()
+        ref_o, ref_l = _oracle(q, cu_q, kc, vc, cache_lens, hq, hkv, scale, True)
+        compare(out, lse, ref_o, ref_l)
+    del kn
+
+
 def test_decode_split_count_changes_only_rounding_and_is_deterministic():
     lq, cache_lens = [1] * 6, [4000, 3000, 1, 2222, 4096, 100]
     cu_q, q, kc, vc, cs, _, _ = _case(9, lq, cache_lens, 4096, 32, 8, 128, False)
