@@ -180,8 +180,8 @@ int varlen_attn_fwd_f32(const float* q, const float* k, const float* v,
  *     library holds until the process exits. It calls no cudaMalloc,
  *     cudaFree or other allocating routine; the caller still owns q/k/v,
  *     the biases, out and lse.
- *   - At most 16384 (sequence, q-block group) pairs: batch *
- *     ceil(max_seqlen_q / 128) when n_heads / n_kv_heads >= 2, batch *
+ *   - At most 16384 work-list pairs: batch * ceil(G * ceil(max_seqlen_q /
+ *     128) / 2) with G = n_heads / n_kv_heads >= 2, batch *
  *     ceil(ceil(max_seqlen_q / 128) / 2) otherwise. Larger problems return
  *     VARLEN_ATTN_ERR_SCRATCH_LIMIT before anything is launched.
  *   - The first call on a device looks up that array's device address (with

@@ -199,8 +199,8 @@ __device__ __forceinline__ Item decode_item(int w, const AttnParams& p) {
   it.Lq = p.cu_q[i + 1] - q0;
   it.Lk = p.cu_k[i + 1] - k0;
   it.kv_row0 = k0;
-  it.kvh = p.pairing == kPairHeads ? hg / p.n_hp : hg / p.group;
-  fill_slots(it, g, hg, p.pairing, p.group, p.n_hp, p.causal);
+  it.kvh = p.pairing == kPairHeads ? hg : hg / p.group;
+  fill_slots(it, g, hg, p.pairing, p.group, p.causal);
   it.q_row0[0] = q0 + it.q_loc0[0];
   it.q_row0[1] = q0 + it.q_loc0[1];
   return it;

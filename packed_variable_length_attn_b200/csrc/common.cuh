@@ -13,8 +13,12 @@ constexpr int kErrBadSeqlens = 9;
 constexpr int kErrTimeout = 10;
 
 // How the two 128-row slots of a CTA work item are filled.
-//  kPairHeads:   two query heads of one K/V group at the same q-block (GQA:
-//                both slots read the same K/V tiles).
+//  kPairHeads:   GQA (G >= 2). The G x (q-blocks) units (q-block, query head)
+//                of one sequence and K/V head, taken q-block by q-block, are
+//                paired consecutively: with G even, two heads at the same
+//                q-block; with G odd, a q-block's last head shares an item
+//                with the next q-block's first one. Both slots read the same
+//                K/V tiles.
 //  kPairQBlocks: two consecutive q-blocks of one head (no GQA sharing).
 constexpr int kPairHeads = 0;
 constexpr int kPairQBlocks = 1;
@@ -34,6 +38,7 @@ struct SchedParams {
   int batch, total_q, total_k, max_q, max_k;
   int causal;
   int pairing;      // kPairHeads / kPairQBlocks; -1 = validate only
+  int group;        // G = Hq / Hkv
   int n_hg;         // work items per (sequence, group) pair
   Workspace ws;
   int* error;       // device error word
@@ -44,7 +49,7 @@ struct AttnParams {
   const int* cu_k;
   int total_q;
   int n_heads, n_kv_heads, group;  // Hq, Hkv, G = Hq / Hkv
-  int pairing, n_hp, n_hg;
+  int pairing, n_hg;
   int causal;
   float scale_log2;                // softmax_scale * log2(e)
   float scale;                     // softmax_scale
@@ -94,22 +99,37 @@ __host__ __device__ __forceinline__ int slot_tiles(int q_loc0, int rows, int Lq,
   return n < nk ? n : nk;
 }
 
-// Number of (sequence, group) pairs sequence i contributes.
-__host__ __device__ __forceinline__ int seq_groups(int Lq, int pairing) {
+// Number of (sequence, group) pairs sequence i contributes: unit pairs of
+// its (q-block, head) units per K/V head, or q-block pairs.
+__host__ __device__ __forceinline__ int seq_groups(int Lq, int pairing, int group) {
   const int nqb = ceil_div(Lq, BM);
-  return pairing == kPairHeads ? nqb : ceil_div(nqb, 2);
+  return pairing == kPairHeads ? ceil_div(group * nqb, 2) : ceil_div(nqb, 2);
+}
+
+// First local query row of slot s of pair g, and the slot's query head
+// (local to the K/V group for kPairHeads).
+__host__ __device__ __forceinline__ void slot_unit(int g, int s, int pairing, int group,
+                                                   int& q_loc0, int& hl) {
+  if (pairing == kPairHeads) {
+    const int unit = 2 * g + s;
+    q_loc0 = (unit / group) * BM;
+    hl = unit % group;
+  } else {
+    q_loc0 = (2 * g + s) * BM;
+    hl = 0;
+  }
 }
 
 __device__ __forceinline__ void fill_slots(Item& it, int g, int hg, int pairing, int group,
-                                           int n_hp, int causal) {
+                                           int causal) {
 #pragma unroll
   for (int s = 0; s < 2; ++s) {
     int active, head, q_loc0;
     if (pairing == kPairHeads) {
-      const int hl = 2 * (hg % n_hp) + s;
-      active = hl < group;
+      int hl;
+      slot_unit(g, s, pairing, group, q_loc0, hl);
+      active = q_loc0 < it.Lq;
       head = it.kvh * group + hl;
-      q_loc0 = g * BM;
     } else {
       head = hg;
       q_loc0 = (2 * g + s) * BM;

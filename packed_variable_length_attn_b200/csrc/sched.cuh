@@ -15,7 +15,7 @@
 //      counts in that order) and place its (sequence, group) pairs there by
 //      K/V tiles to visit, descending: for a causal mask the work of a
 //      q-block never decreases along the sequence, so the pairs go last
-//      q-block first (a lone last q-block of a q-block pair is put where its
+//      first (a lone last unit of an odd number of units is put where its
 //      work falls); without a mask every full pair has the same work and
 //      they keep stream order;
 //   4. publish the item count and a zeroed fetch counter.
@@ -104,10 +104,12 @@ __device__ __forceinline__ int count_below(const unsigned long long* run, int n,
 }
 
 // Work (K/V tiles over both slots) of pair g of a sequence.
-__device__ __forceinline__ int pair_work(int g, int Lq, int Lk, int pairing, int causal) {
+__device__ __forceinline__ int pair_work(int g, int Lq, int Lk, int pairing, int group,
+                                         int causal) {
   int work = 0;
   for (int s = 0; s < 2; ++s) {
-    const int q_loc0 = pairing == kPairHeads ? g * BM : (2 * g + s) * BM;
+    int q_loc0, hl;
+    slot_unit(g, s, pairing, group, q_loc0, hl);
     int rows = Lq - q_loc0;
     rows = rows < 0 ? 0 : (rows > BM ? BM : rows);
     work += slot_tiles(q_loc0, rows, Lq, Lk, causal);
@@ -222,7 +224,7 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedParams 
     int ng = 0, i = 0;
     if (r < B) {
       i = ord[r].x;
-      ng = seq_groups(p.cu_q[i + 1] - p.cu_q[i], p.pairing);
+      ng = seq_groups(p.cu_q[i + 1] - p.cu_q[i], p.pairing, p.group);
     }
     const int off = carry + block_exclusive_scan(ng, s_warp, &s_total);
     if (r < B) ord[r].y = off;
@@ -246,19 +248,20 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedParams 
     const int2 o = ord[r];
     const int i = o.x;
     const int Lq = p.cu_q[i + 1] - p.cu_q[i], Lk = p.cu_k[i + 1] - p.cu_k[i];
-    const int ng = seq_groups(Lq, p.pairing);
-    // a q-block pair whose second q-block does not exist (the last pair of
-    // an odd number of q-blocks) may do less work than the pairs before it
-    const bool lone = p.pairing == kPairQBlocks && (ceil_div(Lq, BM) & 1);
+    const int ng = seq_groups(Lq, p.pairing, p.group);
+    // a pair whose second unit does not exist (the last pair of an odd
+    // number of units) may do less work than the pairs before it
+    const int units = p.pairing == kPairHeads ? p.group * ceil_div(Lq, BM) : ceil_div(Lq, BM);
+    const bool lone = units & 1;
     const int m = lone ? ng - 1 : ng;  // full pairs: work non-decreasing in g
     int cnt = m;                         // place of the lone pair
     if (lone) {
-      const int e = pair_work(ng - 1, Lq, Lk, p.pairing, p.causal);
+      const int e = pair_work(ng - 1, Lq, Lk, p.pairing, p.group, p.causal);
       if (p.causal) {  // full pairs in descending order: the lone one follows those with more work
         int lo = 0, hi = m;  // first full g with work > e
         while (lo < hi) {
           const int mid = (lo + hi) >> 1;
-          if (pair_work(mid, Lq, Lk, p.pairing, p.causal) > e) hi = mid;
+          if (pair_work(mid, Lq, Lk, p.pairing, p.group, p.causal) > e) hi = mid;
           else lo = mid + 1;
         }
         cnt = m - lo;

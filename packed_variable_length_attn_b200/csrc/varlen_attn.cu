@@ -293,9 +293,9 @@ int fwd_bf16(const void* q, const void* k, const void* v, const int32_t* cu_seql
 
   const int G = n_heads / n_kv_heads;
   const int pairing = G >= 2 ? kPairHeads : kPairQBlocks;
-  const int n_hp = (G + 1) / 2;
-  const int n_hg = pairing == kPairHeads ? n_kv_heads * n_hp : n_heads;
-  const int64_t groups_per_seq = seq_groups(max_seqlen_q, pairing);
+  const int n_hg = pairing == kPairHeads ? n_kv_heads : n_heads;
+  if ((int64_t)G * ceil_div(max_seqlen_q, BM) > INT32_MAX / 2) return VARLEN_ATTN_ERR_TOO_LARGE;
+  const int64_t groups_per_seq = seq_groups(max_seqlen_q, pairing, G);
   const int64_t capacity = (int64_t)batch * groups_per_seq;
   if (capacity * n_hg > INT32_MAX || capacity > (INT32_MAX / 16)) return VARLEN_ATTN_ERR_TOO_LARGE;
 
@@ -333,6 +333,7 @@ int fwd_bf16(const void* q, const void* k, const void* v, const int32_t* cu_seql
   sp.max_k = max_seqlen_k;
   sp.causal = a.causal;
   sp.pairing = pairing;
+  sp.group = G;
   sp.n_hg = n_hg;
   sp.ws = ws;
   sp.error = di->error_word;
@@ -346,7 +347,6 @@ int fwd_bf16(const void* q, const void* k, const void* v, const int32_t* cu_seql
   prm.n_kv_heads = n_kv_heads;
   prm.group = G;
   prm.pairing = pairing;
-  prm.n_hp = n_hp;
   prm.n_hg = n_hg;
   prm.causal = a.causal;
   prm.scale_log2 = softmax_scale * 1.4426950408889634f;

@@ -46,6 +46,8 @@ SMALL = [
     ([1, 1, 1, 1], [513, 1, 128, 129], 7, 1, 64, True),      # decode rows, G = 7
     ([385, 3], [385, 700], 3, 1, 128, False),               # odd G
     ([640], None, 2, 1, 128, True),
+    ([640, 300, 5, 129], None, 7, 1, 64, True),               # odd G: pairs across q-blocks
+    ([200, 333, 1], [500, 333, 40], 5, 1, 128, True),        # odd G, Lq != Lk
 ]
 
 
