@@ -418,6 +418,11 @@ def run_gpu(args, world, rank, local):
             va.set_profile_events()
             cev[i][1].record(stream)
     else:
+        # one pass: the step time over K calls and, in the same calls, the
+        # attention kernel's own time from events the library records around
+        # its launch. (Those events sit between the schedule and attention
+        # launches, so during timing the attention kernel's set-up does not
+        # overlap the schedule kernel as it does in an unprofiled call.)
         t0.record(stream)
         for i in range(args.steps):
             va.set_profile_events(*kev[i])

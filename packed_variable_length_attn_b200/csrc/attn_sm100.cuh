@@ -216,6 +216,9 @@ __device__ void load_role(const Smem<D>& sm, const CUtensorMap* tm_q, const CUte
   using C = KCfg<D>;
   const unsigned FULL = 0xffffffffu;
   uint32_t kv_t = 0, q_uses[2] = {0, 0};
+  // the work list is written by the schedule kernel launched just before
+  // (this kernel may start before it ends: programmatic dependent launch)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int count = *reinterpret_cast<volatile int*>(p.ws.count);
   bool ok = true;
   auto load_kv = [&](const CUtensorMap* tm, int kvh, int row) {
@@ -510,10 +513,18 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
       const uint32_t ph = g & 1;             // phase of s_full / p_full for this tile
       float* bk = nullptr;
       if constexpr (kBiasKey) {
+        // this thread's key's bias into the group's staging row, asynchronously
+        // (the barrier completes when all 128 copies have landed), ahead of
+        // the pair-grid copies so that the two latencies overlap
         bk = sm.bias(wg, b);
         const int key = kb + r;
-        bk[r] = key < Lk ? p.bias_key[(long long)(kv_row0 + key) * p.n_heads + head] : 0.f;
-        ptx::mbar_arrive(sm.bias_full(wg, b));
+        const bool in = key < Lk;
+        ptx::cp_async4_zfill(ptx::smem_u32(bk + r),
+                             in ? p.bias_key + (long long)(kv_row0 + key) * p.n_heads + head
+                                : p.bias_key,
+                             in ? 4u : 0u);
+        ptx::cp_async_mbar_arrive_noinc(sm.bias_full(wg, b));
+        ptx::cp_async_commit_group();
       }
       // Pair grid, 16-byte rows: the warp's 32 rows x 128 keys arrive in
       // chunks of 16 keys (2 KB) through a ring of kPairBufs staging blocks,
@@ -758,7 +769,7 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
       p.lse[(long long)head * p.total_q + q_row0 + r] = lse;
     }
   }
-  if constexpr (kBiasPair) ptx::cp_async_wait_group<0>();  // copies left by an abort
+  if constexpr (kBiasKey || kBiasPair) ptx::cp_async_wait_group<0>();  // copies left by an abort
 }
 
 // ------------------------------------------------------------------ kernel

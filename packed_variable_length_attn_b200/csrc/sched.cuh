@@ -123,6 +123,9 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedParams 
   __shared__ int s_warp[32];
   __shared__ int s_total;
   const int tid = threadIdx.x;
+  // The attention kernel launched after this one may begin its set-up now;
+  // it reads the work list only after this grid has completed.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (tid == 0) s_bad = 0;
   __syncthreads();
 

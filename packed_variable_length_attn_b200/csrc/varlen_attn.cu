@@ -221,7 +221,23 @@ int launch_attn(int grid, const CUtensorMap& tq, const CUtensorMap& tk, const CU
     if (int rc = set_smem(kern, KCfg<D>::kSmemBytes)) return rc;
     configured_for = dev;
   }
-  kern<<<grid, kAttnThreads, KCfg<D>::kSmemBytes, st>>>(tq, tk, tv, prm);
+  // Programmatic dependent launch: the kernel may start while the schedule
+  // kernel before it on the stream still runs (its barrier set-up, tensor
+  // memory allocation and descriptor prefetch overlap it); the load warp
+  // waits for the schedule kernel's results (griddepcontrol.wait) before it
+  // reads the work list, and no other role reads what the schedule writes.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kAttnThreads);
+  cfg.dynamicSmemBytes = KCfg<D>::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, prm);
+  if (e != cudaSuccess) return cuda_fail("launch attn_fwd_sm100", e);
   return check_launch("launch attn_fwd_sm100");
 }
 
