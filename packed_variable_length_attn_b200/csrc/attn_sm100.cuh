@@ -730,20 +730,24 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
     const uint32_t stg = ptx::smem_u32(sm.epi(warp));
     auto unit_addr = [&](int x, int c) { return stg + (uint32_t)(4 * x + (c ^ ((x >> 1) & 3))) * 16u; };
     const int wrow0 = (warp & 3) * 32;  // first tile row of this warp
+    // all of this row's O columns from tensor memory, then one wait
+    uint32_t o[D];
+    if (n > 0) {
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c)
+        ptx::tmem_ld32(t_o + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[c * 32]));
+      ptx::tmem_wait_ld();
+    } else {
+#pragma unroll
+      for (int e = 0; e < D; ++e) o[e] = 0u;
+    }
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
-      uint32_t o[32];
-      if (n > 0) {
-        ptx::tmem_ld32(t_o + c * 32, o);
-        ptx::tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = 0u;
-      }
       uint32_t vw[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e)
-        vw[e] = ptx::pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+        vw[e] = ptx::pack_bf16x2(__uint_as_float(o[c * 32 + 2 * e]) * inv,
+                                 __uint_as_float(o[c * 32 + 2 * e + 1]) * inv);
       __syncwarp();  // the previous block's reads are done
 #pragma unroll
       for (int u4 = 0; u4 < 4; ++u4)

@@ -410,6 +410,12 @@ constexpr int kDec2Consumers = 4;
 constexpr int kDec2Threads = 32 * (kDec2Consumers + 1);
 constexpr int kDec2Stages = 4;
 constexpr int kDec2MaxRows = 8;
+// Block t goes to stage t % kDec2Stages and consumer warp t % kDec2Consumers.
+// A consumer reaches block t only after block t - kDec2Consumers, so with at
+// least as many stages as consumers the stage's previous fill (block
+// t - kDec2Stages) has already landed and a parity wait can never match an
+// older phase of the barrier.
+static_assert(kDec2Consumers <= kDec2Stages, "a consumer must never run two fills ahead");
 
 template <int D, int RT>
 struct Dec2Cfg {
