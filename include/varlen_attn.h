@@ -79,7 +79,8 @@ typedef enum varlen_attn_status {
  * Runs on tensor cores (tcgen05, accumulators in tensor memory).
  *
  *   q        [total_q, n_heads, head_dim] bf16, contiguous, 16-byte aligned.
- *   k, v     [total_k, n_kv_heads, head_dim] bf16, contiguous, 16-byte aligned.
+ *   k, v     [total_k, n_kv_heads, head_dim] bf16, contiguous, 16-byte aligned
+ *            (may be NULL when total_k is 0: no row then sees a key).
  *   cu_seqlens_q, cu_seqlens_k
  *            [batch + 1] int32 device arrays; sequence i owns query rows
  *            [cu_q[i], cu_q[i+1]) and key rows [cu_k[i], cu_k[i+1]).
@@ -221,7 +222,8 @@ int varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v,
  *   dout [total_q, n_heads, head_dim] bf16: the gradient of the loss w.r.t. out.
  * Outputs (caller-owned, written, not accumulated):
  *   dq [total_q, n_heads, head_dim], dk and dv [total_k, n_kv_heads, head_dim]
- *   bf16 (dk, dv summed over the n_heads / n_kv_heads query heads of a group);
+ *   bf16 (dk, dv summed over the n_heads / n_kv_heads query heads of a group;
+ *   k, v, dk and dv may be NULL when total_k is 0);
  *   dbias_per_key [total_k, n_heads] fp32 or NULL (not computed);
  *   dbias_pair fp32 or NULL: entry (i, h, r, c) at i*dbias_stride_b +
  *   h*dbias_stride_h + r*dbias_stride_q + c for every query head h and every

@@ -161,6 +161,13 @@ bool make_tmap(CUtensorMap* m, const void* base, int D, int heads, int rows, int
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// Base of a K or V tensor map. With no keys at all (total_k == 0, k and v
+// possibly NULL) no K/V tile is ever loaded, but a tensor map still needs a
+// valid aligned address: q's stands in.
+const void* kv_base(const void* kv, const void* q, int total_k) {
+  return total_k > 0 ? kv : q;
+}
+
 struct Common {
   int batch, total_q, total_k, max_q, max_k, Hq, Hkv, D, causal;
   const int32_t *cu_q, *cu_k;
@@ -170,7 +177,9 @@ struct Common {
 
 int validate_common(const Common& a, const void* q, const void* k, const void* v, const void* out,
                     const float* lse) {
-  if (!q || !k || !v || !out || !a.cu_q || !a.cu_k) return VARLEN_ATTN_ERR_NULL_POINTER;
+  if (!q || !out || !a.cu_q || !a.cu_k) return VARLEN_ATTN_ERR_NULL_POINTER;
+  // k and v may be NULL only when there are no keys at all (never read then)
+  if (a.total_k > 0 && (!k || !v)) return VARLEN_ATTN_ERR_NULL_POINTER;
   if (a.batch <= 0 || a.Hq <= 0 || a.Hkv <= 0 || a.D <= 0 || a.total_q < 0 || a.total_k < 0 ||
       a.max_q < 0 || a.max_k < 0)
     return VARLEN_ATTN_ERR_BAD_SHAPE;
@@ -335,8 +344,8 @@ int fwd_bf16(const void* q, const void* k, const void* v, const int32_t* cu_seql
 
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, q, head_dim, n_heads, total_q, BM) ||
-      !make_tmap(&tk, k, head_dim, n_kv_heads, total_k, BN) ||
-      !make_tmap(&tv, v, head_dim, n_kv_heads, total_k, BN))
+      !make_tmap(&tk, kv_base(k, q, total_k), head_dim, n_kv_heads, total_k, BN) ||
+      !make_tmap(&tv, kv_base(v, q, total_k), head_dim, n_kv_heads, total_k, BN))
     return VARLEN_ATTN_ERR_CUDA;
 
   SchedParams sp;
@@ -843,7 +852,8 @@ int varlen_attn_bwd(const void* q, const void* k, const void* v, const void* out
            bias_stride_h, bias_stride_q, bias_stride_k};
   int rc = validate_common(a, q, k, v, out, lse);
   if (rc) return rc;
-  if (!lse || !dout || !dq || !dk || !dv) return VARLEN_ATTN_ERR_NULL_POINTER;
+  if (!lse || !dout || !dq) return VARLEN_ATTN_ERR_NULL_POINTER;
+  if (total_k > 0 && (!dk || !dv)) return VARLEN_ATTN_ERR_NULL_POINTER;
   if (!aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
       (dbias_per_key && !aligned(dbias_per_key, 4)) || (dbias_pair && !aligned(dbias_pair, 4)))
     return VARLEN_ATTN_ERR_MISALIGNED;
@@ -894,8 +904,8 @@ int varlen_attn_bwd(const void* q, const void* k, const void* v, const void* out
   CUtensorMap tq, tk, tv, tdo;
   if (!make_tmap(&tq, q, head_dim, n_heads, total_q, BM) ||
       !make_tmap(&tdo, dout, head_dim, n_heads, total_q, BM) ||
-      !make_tmap(&tk, k, head_dim, n_kv_heads, total_k, BN) ||
-      !make_tmap(&tv, v, head_dim, n_kv_heads, total_k, BN))
+      !make_tmap(&tk, kv_base(k, q, total_k), head_dim, n_kv_heads, total_k, BN) ||
+      !make_tmap(&tv, kv_base(v, q, total_k), head_dim, n_kv_heads, total_k, BN))
     return VARLEN_ATTN_ERR_CUDA;
 
   if (dbias_per_key) {  // the dK/dV kernel adds two half sums per (key, head)

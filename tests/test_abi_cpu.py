@@ -64,6 +64,10 @@ def test_host_validation_codes(lib):
     # the pointer values are never dereferenced: validation fails first
     assert _call(lib, q=None) == 1
     assert _call(lib, cu_k=None) == 1
+    assert _call(lib, k=None) == 1          # keys exist: k and v are required
+    assert _call(lib, v=None) == 1
+    if not torch.cuda.is_available():       # with no keys NULL k/v pass validation
+        assert _call(lib, k=None, v=None, total_k=0, max_k=0) == 7
     assert _call(lib, batch=0) == 2
     assert _call(lib, hq=0) == 2
     assert _call(lib, total_q=-1) == 2
@@ -156,6 +160,9 @@ def test_backward_host_validation_codes(lib):
     assert call(lse=None) == 1
     assert call(dout=None) == 1
     assert call(dk=None) == 1
+    assert call(dv=None) == 1
+    if not torch.cuda.is_available():       # with no keys dK/dV are never written
+        assert call(k=None, v=None, dk=None, dv=None, tk=0, mk=0) == 7
     assert call(batch=0) == 2
     assert call(hq=6, hkv=4) == 3
     assert call(d=96) == 4
