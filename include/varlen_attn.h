@@ -272,11 +272,14 @@ int varlen_attn_bwd(const void* q, const void* k, const void* v, const void* out
  *   max_seqlen_q * (n_heads / n_kv_heads) <= 32 (decode-sized queries; longer
  *   ones belong to varlen_attn_fwd): else VARLEN_ATTN_ERR_BAD_SHAPE.
  *   out [total_q, n_heads, head_dim] bf16, lse [n_heads, total_q] fp32 or NULL.
- *   num_splits: key splits per (sequence, K/V head); 0 = chosen from the batch
- *            size and cache_len. With more than one split, partial results go
- *            to the library workspace and a third launch merges them; results
- *            depend on the split count in the last bits (the merge order), so
- *            give a fixed num_splits where bitwise reproducibility across batch
+ *   num_splits: the cache's key positions are cut into num_splits equal
+ *            ranges (whole 32-key blocks; ranges past a sequence's length are
+ *            empty and cost one short CTA), one CTA per (range, K/V head,
+ *            sequence); 0 = chosen from the batch size and cache_len (ranges of
+ *            at most 1536 keys). With more than one range, partial results go to
+ *            the library workspace and a third launch merges them; results
+ *            depend on the ranges in the last bits (the merge order), so give a
+ *            fixed num_splits where bitwise reproducibility across batch
  *            compositions matters.
  * HBM-bound (every cached key and value is read once): fp32 on the CUDA
  * cores, no bias. Errors as for varlen_attn_fwd; a cache position beyond

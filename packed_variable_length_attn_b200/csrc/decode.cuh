@@ -39,6 +39,7 @@ struct DecodeParams {
   const __nv_bfloat16* k_new;   // [Tq, Hkv, D] or null
   const __nv_bfloat16* v_new;
   int batch, total_q, cache_len, n_heads, n_kv_heads, group, causal, n_splits;
+  int split_blocks;             // key blocks per split, the same for every sequence
   float scale_log2;             // softmax_scale * log2(e)
   __nv_bfloat16* out;           // [Tq, Hq, D]
   float* lse;                   // [Hq, Tq] or null
@@ -61,6 +62,23 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Key blocks [b0, b1) of split `split` of a sequence with nblk_all blocks: the
+// splits are fixed ranges of the cache (split_blocks blocks each), so a split
+// costs the same in every sequence and the shorter sequences leave their last
+// splits empty. An empty split (with more than one split) only marks its rows'
+// partial LSE as -inf, which the combine skips.
+__device__ __forceinline__ bool split_range(const DecodeParams& p, int split, int nblk_all, int q0,
+                                            int R, int g, int& b0, int& b1) {
+  b0 = split * p.split_blocks;
+  b1 = min(nblk_all, b0 + p.split_blocks);
+  if (b1 > b0 || p.n_splits == 1) return true;
+  for (int rho = threadIdx.x; rho < R; rho += blockDim.x) {
+    const int r = rho / p.group, h = g * p.group + (rho - r * p.group);
+    p.part_lse[(long long)split * p.n_heads * p.total_q + (long long)h * p.total_q + q0 + r] = -INFINITY;
+  }
+  return false;
+}
 
 // Writes the new K/V rows of every sequence into its cache rows
 // [cache_seqlens[i], cache_seqlens[i] + Lq_i); 16-byte units, grid-stride.
@@ -144,8 +162,8 @@ __global__ void __launch_bounds__(kDecThreads, RT <= 8 ? 4 : 2) decode_kernel(De
   }
   // this split's keys, in whole blocks
   const int nblk_all = (Lk + kDecKeys - 1) / kDecKeys;
-  const int per = (nblk_all + p.n_splits - 1) / p.n_splits;
-  const int b0 = split * per, b1 = min(nblk_all, b0 + per);
+  int b0, b1;
+  if (!split_range(p, split, nblk_all, q0, R, g, b0, b1)) return;
 
   for (int e = tid; e < RT * D; e += kDecThreads) {
     const int rho = e / D, d = e - rho * D;
@@ -370,6 +388,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_combine_kernel(DecodeParam
     if (mx != -INFINITY) {
       for (int s = 0; s < p.n_splits; ++s) {
         const float ls = p.part_lse[(long long)s * p.n_heads * p.total_q + (long long)h * p.total_q + t];
+        if (ls == -INFINITY) continue;  // an empty split (its O was never written)
         const float wgt = __expf(ls - mx);
         wsum += wgt;
         const float* po = p.part_o + ((long long)s * p.total_q * p.n_heads + e) * D;
@@ -461,8 +480,8 @@ __global__ void __launch_bounds__(kDec2Threads) decode_tma_kernel(
     return;
   }
   const int nblk_all = (Lk + kDecKeys - 1) / kDecKeys;
-  const int per = (nblk_all + p.n_splits - 1) / p.n_splits;
-  const int b0 = split * per, b1 = min(nblk_all, b0 + per);
+  int b0, b1;
+  if (!split_range(p, split, nblk_all, q0, R, g, b0, b1)) return;
   const int nblk = max(0, b1 - b0);
 
   if (tid == 0) {

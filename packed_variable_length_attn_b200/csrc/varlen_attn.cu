@@ -722,17 +722,26 @@ int varlen_attn_decode(const void* q, const int32_t* cu_seqlens_q, int batch, in
   if (int rc = device_info(&di)) return rc;
   if (total_q == 0 || max_seqlen_q == 0) return VARLEN_ATTN_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // splits: about 16 CTAs per SM over the whole grid (several waves keep the
-  // SMs busy despite unequal cache lengths), each split at least 256 keys
+  // splits: fixed ranges of split_blocks key blocks of the cache, so that
+  // every CTA streams about the same number of keys whatever its sequence's
+  // length (the grid then ends without a tail of long CTAs). Automatic count:
+  // splits of at most 1536 keys (smaller ones measured slower: each CTA's
+  // set-up, merge and partial output cost more than the shorter tail saves),
+  // and about 16 CTAs per SM over the whole grid when that asks for more,
+  // each split at least 256 keys.
   int splits = num_splits;
   const int max_blocks = (cache_len + kDecKeys - 1) / kDecKeys;
   if (splits == 0) {
     const int64_t ctas = (int64_t)batch * n_kv_heads;
     const int64_t want = (16 * (int64_t)di->sm_count + ctas - 1) / ctas;
+    const int64_t by_size = (max_blocks + 1536 / kDecKeys - 1) / (1536 / kDecKeys);
     const int min_blocks = (256 + kDecKeys - 1) / kDecKeys;
-    splits = (int)std::max<int64_t>(1, std::min<int64_t>(want, std::max(1, max_blocks / min_blocks)));
+    splits = (int)std::max<int64_t>(
+        1, std::min<int64_t>(std::max(want, by_size), std::max(1, max_blocks / min_blocks)));
   }
   splits = std::min(splits, std::max(1, max_blocks));
+  const int split_blocks = (max_blocks + splits - 1) / splits;
+  splits = (max_blocks + split_blocks - 1) / split_blocks;  // no split starts past the cache
   DecodeParams dp;
   dp.q = static_cast<const __nv_bfloat16*>(q);
   dp.cu_q = cu_seqlens_q;
@@ -749,6 +758,7 @@ int varlen_attn_decode(const void* q, const int32_t* cu_seqlens_q, int batch, in
   dp.group = G;
   dp.causal = causal ? 1 : 0;
   dp.n_splits = splits;
+  dp.split_blocks = split_blocks;
   dp.scale_log2 = softmax_scale * 1.4426950408889634f;
   dp.out = static_cast<__nv_bfloat16*>(out);
   dp.lse = lse;
