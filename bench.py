@@ -442,41 +442,88 @@ def run_gpu(args, world, rank, local):
     if va.get_device_error() != 0:
         raise RuntimeError("device error during the timed region")
 
-    # ---- end to end through host buffers (pinned), copies inside the region
+    # ---- end to end through host buffers (pinned), copies inside the region.
+    # Every step copies its inputs host -> device, runs the call and reads its
+    # output and LSE back to the host. Steps are pipelined the way a serving
+    # loop would run them: two sets of device buffers, the input copies on one
+    # copy stream and the output copies on another, so step k + 1's inputs
+    # travel while step k computes and step k - 1's results come back (each
+    # direction of the host link busy on its own).
     hq, hk, hv = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
     hcq, hck = cu_q.cpu().pin_memory(), cu_k.cpu().pin_memory()
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    dq, dk_, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    dcq, dck = torch.empty_like(cu_q), torch.empty_like(cu_k)
+    hbias = {key: t.cpu().pin_memory() for key, t in
+             (("bias_per_key", bias_kw["bias_per_key"]), ("bias_pair", bias_kw["bias_pair"]))
+             if t is not None}
+    n_buf = 2
+    hout = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(n_buf)]
+    hlse = [torch.empty(lse.shape, dtype=lse.dtype).pin_memory() for _ in range(n_buf)]
+    dbuf = [dict(q=torch.empty_like(q), k=torch.empty_like(k), v=torch.empty_like(v),
+                 cq=torch.empty_like(cu_q), ck=torch.empty_like(cu_k), out=torch.empty_like(out),
+                 lse=torch.empty_like(lse),
+                 **{key: torch.empty_like(bias_kw[key]) for key in hbias})
+            for _ in range(n_buf)]
+    h2d_stream = torch.cuda.Stream(device=dev)
+    d2h_stream = torch.cuda.Stream(device=dev)
+    computed = [None] * n_buf   # event: the call of the buffer set's last step is done
+    read_back = [None] * n_buf  # event: its output has been copied to the host
 
-    def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk_.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        dcq.copy_(hcq, non_blocking=True)
-        dck.copy_(hck, non_blocking=True)
-        va.varlen_attn_fwd(dq, dk_, dv, dcq, dck, w.max_seqlen_q, w.max_seqlen_k,
-                           softmax_scale=w.softmax_scale, causal=w.causal, out=out, lse=lse,
-                           **bias_kw)
-        hout.copy_(out, non_blocking=True)
-        hlse.copy_(lse, non_blocking=True)
+    def e2e_step(kstep):
+        b = kstep % n_buf
+        d = dbuf[b]
+        with torch.cuda.stream(h2d_stream):
+            if computed[b] is not None:
+                h2d_stream.wait_event(computed[b])   # inputs of set b no longer read
+            d["q"].copy_(hq, non_blocking=True)
+            d["k"].copy_(hk, non_blocking=True)
+            d["v"].copy_(hv, non_blocking=True)
+            d["cq"].copy_(hcq, non_blocking=True)
+            d["ck"].copy_(hck, non_blocking=True)
+            for key, t in hbias.items():
+                d[key].copy_(t, non_blocking=True)
+            loaded = torch.cuda.Event()
+            loaded.record(h2d_stream)
+        stream.wait_event(loaded)
+        if read_back[b] is not None:
+            stream.wait_event(read_back[b])          # output of set b copied out
+        va.varlen_attn_fwd(d["q"], d["k"], d["v"], d["cq"], d["ck"], w.max_seqlen_q,
+                           w.max_seqlen_k, softmax_scale=w.softmax_scale, causal=w.causal,
+                           out=d["out"], lse=d["lse"], stream=stream,
+                           bias_per_key=d.get("bias_per_key"), bias_pair=d.get("bias_pair"),
+                           bias_pair_strides=bias_kw["bias_pair_strides"])
+        done = torch.cuda.Event()
+        done.record(stream)
+        computed[b] = done
+        with torch.cuda.stream(d2h_stream):
+            d2h_stream.wait_event(done)
+            hout[b].copy_(d["out"], non_blocking=True)
+            hlse[b].copy_(d["lse"], non_blocking=True)
+            rb = torch.cuda.Event()
+            rb.record(d2h_stream)
+        read_back[b] = rb
 
-    e2e_step()
+    e2e_step(0)
     torch.cuda.synchronize()
+    if not (torch.equal(hout[0].view(torch.int16), out.cpu().view(torch.int16))):
+        raise RuntimeError("end-to-end output differs from the device-timed output")
     e_steps = max(1, min(args.steps, args.e2e_steps))
     if world > 1:
         dist.barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e_steps):
-        e2e_step()
+    h2d_stream.wait_event(e0)
+    computed = [None] * n_buf
+    read_back = [None] * n_buf
+    for kstep in range(e_steps):
+        e2e_step(kstep)
+    for ev in read_back:
+        if ev is not None:
+            stream.wait_event(ev)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e_steps
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcq, hck))
-    d2h = hout.numel() * hout.element_size() + hlse.numel() * hlse.element_size()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcq, hck, *hbias.values()))
+    d2h = hout[0].numel() * hout[0].element_size() + hlse[0].numel() * hlse[0].element_size()
 
     # ---- reduce over ranks
     (elapsed_ms, e2e_ms, kern_ms), (all_flops, all_tokens) = reduce_over_ranks(
