@@ -109,6 +109,11 @@ typedef enum varlen_attn_status {
  *            outside every sequence (beyond cu_q[B]) are not written.
  *   lse      NULL, or [n_heads, total_q] fp32 output: natural-log sum of exp of
  *            the scaled, biased scores (-inf for a row that sees no key).
+ * Inputs are taken to be finite. A sequence's last key tile (128 rows) may
+ * reach into the next sequence's rows, whose probabilities are exactly 0, so
+ * an Inf or NaN in a neighbour's V would reach this sequence through 0 * Inf;
+ * with finite inputs every sequence's results are independent of its
+ * neighbours bit for bit.
  */
 int varlen_attn_fwd(const void* q, const void* k, const void* v,
                     const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
