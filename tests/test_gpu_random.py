@@ -6,8 +6,10 @@ in both directions), the GQA group, head_dim, the mask, and the biases
 (per-key, per-pair grid shared by the heads, per query head or per K/V head),
 then compares every output element of the CUDA path (through the C ABI) with
 the oracle at the library's tolerances. The same draws feed the backward (all
-gradients) and the K/V-cache decode step. Sizes stay small enough for the
-fp64 oracle to finish each case in well under a second.
+gradients) and the K/V-cache decode step; random masks and row shapes feed the
+unpad / pad helpers (bit for bit) and random strided grids the first-token
+fold. Sizes stay small enough for the fp64 oracle to finish each case in well
+under a second.
 """
 import numpy as np
 import pytest
@@ -211,3 +213,81 @@ def test_random_decode(seed):
     cu_k = torch.tensor(np.concatenate([[0], np.cumsum(lk)]), dtype=torch.int32)
     ref_o, ref_l = oracle.fwd(q, k, v, cu_q, cu_k, Hq, Hkv, scale, True)
     compare(out, lse, ref_o, ref_l)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_random_unpad_pad_bit_exact(seed):
+    """Random masks (holes, prefixes, empty and full rows) and row shapes:
+    unpadding metadata, gather and scatter bit for bit against the oracle."""
+    r = np.random.default_rng(7000 + seed)
+    B, S = int(r.integers(1, 10)), int(r.integers(1, 700))
+    kind = int(r.integers(0, 3))
+    if kind == 0:
+        mask = r.random((B, S)) < r.uniform(0.05, 0.95)
+    else:
+        mask = np.zeros((B, S), dtype=bool)
+        for b in range(B):
+            L = int(r.integers(0, S + 1))
+            mask[b, :L] = True
+        if kind == 2:  # and a few holes
+            mask &= r.random((B, S)) < 0.9
+    H = int(r.choice([1, 2, 3, 8]))
+    D = int(r.choice([8, 64, 128]))
+    dtype = torch.bfloat16 if r.integers(0, 2) else torch.float32
+    g = torch.Generator().manual_seed(8000 + seed)
+    x = torch.randn(B, S, H, D, generator=g).to(dtype)
+    packed, idx, cu, mx = va.unpad(x.cuda(), torch.from_numpy(mask).cuda())
+    back = va.pad(packed, idx, cu, B, S)
+    torch.cuda.synchronize()
+    ref_cu, ref_idx, ref_mx = layout.mask_to_seqlens(mask)
+    assert cu.cpu().numpy().tolist() == ref_cu.tolist()
+    assert int(mx) == ref_mx
+    bits = torch.int16 if dtype == torch.bfloat16 else torch.int32
+    rows = x.view(bits).numpy().reshape(B * S, H, D)
+    ref_packed = layout.gather_rows(rows, ref_idx)
+    assert np.array_equal(packed.cpu().view(bits).numpy(), ref_packed)
+    ref_back = layout.scatter_rows(ref_packed, ref_idx, B * S).reshape(B, S, H, D)
+    assert np.array_equal(back.cpu().view(bits).numpy(), ref_back)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_fold_matches_oracle(seed):
+    """First-token fold of random strided grids (per query head or per K/V
+    head, with and without a per-key bias to add to)."""
+    r = np.random.default_rng(9000 + seed)
+    B = int(r.integers(1, 9))
+    lk = [int(x) for x in r.integers(0, 300, B)]
+    if sum(lk) == 0:
+        lk[0] = 1
+    Hkv = int(r.choice([1, 2, 4]))
+    G = int(r.choice([1, 2, 4]))
+    Hq = Hkv * G
+    kv_heads = bool(r.integers(0, 2))
+    Hg = Hkv if kv_heads else Hq
+    rows = int(r.integers(1, 4))
+    row = int(r.integers(0, rows))
+    with_key = bool(r.integers(0, 2))
+    w = workloads.make_custom([1] * B, lk, n_heads=Hq, n_kv_heads=Hkv, head_dim=64, causal=False,
+                              seed=9100 + seed, bias_pair=(B, Hg, rows, max(lk)),
+                              bias_key=with_key)
+    dev = to_device(w)
+    head_div = G if kv_heads else 1
+    folded = va.fold_pair_bias_row(dev["bias_pair"], dev["cu_k"], Hq, w.total_k, row=row,
+                                   head_div=head_div,
+                                   bias_in=dev["bias_key"] if with_key else None)
+    torch.cuda.synchronize()
+    gflat = w.bias_pair.numpy().reshape(-1)
+    sb, sh, sr, sc = w.bias_strides
+    cu = w.cu_k.numpy()
+    want = np.zeros((w.total_k, Hq), dtype=np.float32)
+    for i in range(B):
+        for h in range(Hq):
+            for c in range(lk[i]):
+                v = np.float32(gflat[i * sb + (h // head_div) * sh + row * sr + c * sc])
+                want[cu[i] + c, h] = (np.float32(w.bias_key[cu[i] + c, h].item()) + v
+                                      if with_key else v)
+    assert np.array_equal(folded.cpu().numpy(), want)
+    ref = layout.fold_pair_row(w.bias_pair.numpy(), w.bias_strides, row, cu, Hq, w.total_k,
+                               head_div=head_div,
+                               bias_key=w.bias_key.numpy() if with_key else None)
+    np.testing.assert_allclose(folded.cpu().numpy(), ref, rtol=1e-6, atol=1e-6)
