@@ -326,6 +326,8 @@ def _config(w, args=None):
          "total_tokens": w.total_q, "n_heads": w.n_heads, "n_kv_heads": w.n_kv_heads,
          "head_dim": w.head_dim, "causal": w.causal, "bias": BIAS.get(cfg),
          "useful_pairs_per_head": pairs, "seed": w.meta.get("seed"), "l2": l2}
+    if getattr(args, "graph", False):
+        d["launch"] = "CUDA graph replay of the captured step"
     if w.batch <= 64:
         d["lengths_drawn"] = list(w.lengths_q)
     return d
@@ -389,6 +391,25 @@ def run_gpu(args, world, rank, local):
     torch.cuda.synchronize()
     if va.get_device_error() != 0:
         raise RuntimeError("device error during warm-up")
+    graph = None
+    if args.graph:
+        # the step captured once in a CUDA graph (after a warm-up call on the
+        # capture stream, which sizes the library's workspace there) and
+        # replayed: no host work per step
+        cap = torch.cuda.Stream(device=dev)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            step()
+        stream.wait_stream(cap)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            step()
+        for _ in range(max(3, args.warmup)):
+            graph.replay()
+        torch.cuda.synchronize()
+        if va.get_device_error() != 0:
+            raise RuntimeError("device error during graph warm-up")
 
     # ---- timed region: K steps, device events, per-launch kernel events
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -413,9 +434,14 @@ def run_gpu(args, world, rank, local):
         for i in range(args.steps):
             scrub.fill_(float(i))
             cev[i][0].record(stream)
-            va.set_profile_events(*kev[i])
-            step()
-            va.set_profile_events()
+            if graph is not None:
+                kev[i][0].record(stream)
+                graph.replay()
+                kev[i][1].record(stream)
+            else:
+                va.set_profile_events(*kev[i])
+                step()
+                va.set_profile_events()
             cev[i][1].record(stream)
     else:
         # one pass: the step time over K calls and, in the same calls, the
@@ -424,10 +450,17 @@ def run_gpu(args, world, rank, local):
         # launches, so during timing the attention kernel's set-up does not
         # overlap the schedule kernel as it does in an unprofiled call.)
         t0.record(stream)
-        for i in range(args.steps):
-            va.set_profile_events(*kev[i])
-            step()
-        va.set_profile_events()
+        if graph is not None:
+            # per-step events around each replay (schedule + attention kernel)
+            for i in range(args.steps):
+                kev[i][0].record(stream)
+                graph.replay()
+                kev[i][1].record(stream)
+        else:
+            for i in range(args.steps):
+                va.set_profile_events(*kev[i])
+                step()
+            va.set_profile_events()
         t1.record(stream)
     torch.cuda.synchronize()
     sampler.mark_stop()
@@ -563,6 +596,8 @@ def run_gpu(args, world, rank, local):
         rl["kernel"] = (f"attn_fwd_sm100<{w.head_dim},{str(w.bias_key is not None).lower()},"
                         f"{str(w.bias_pair is not None).lower()}>")
         rl["kernel_ms_per_launch"] = kern_ms
+        if args.graph:
+            rl["kernel_ms_covers"] = "one graph replay: schedule and attention kernels"
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
@@ -798,6 +833,9 @@ def main():
                     help="--impl reference: seconds of oracle work over all steps")
     ap.add_argument("--config", type=int, default=WORKLOAD, choices=[1, 2, 3, 4, 5],
                     help="named workload (default: the long causal GQA workload)")
+    ap.add_argument("--graph", action="store_true",
+                    help="time CUDA-graph replays of the captured step (no host work per step); "
+                         "the per-launch time then covers the schedule and attention kernels")
     ap.add_argument("--flush-l2", action="store_true",
                     help="256 MB scrub write between timed steps; each call timed alone")
     ap.add_argument("--decode", action="store_true",
