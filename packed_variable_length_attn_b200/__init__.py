@@ -23,6 +23,9 @@ helpers) and ``fold_pair_bias_row`` (first-token bias fold).
     dq, dk, dv, _, _ = varlen_attn_bwd(q, k, v, out, lse, dout, cu_seqlens_q,
                                        cu_seqlens_k, max_seqlen_q, max_seqlen_k,
                                        causal=True)
+
+``varlen_attn`` wraps the two in a ``torch.autograd.Function`` for training
+loops (bf16; gradients for q, k, v and the biases that require them).
 """
 from __future__ import annotations
 
@@ -35,7 +38,7 @@ __all__ = ["varlen_attn_fwd", "varlen_attn_fwd_noalloc", "library_path", "load_l
            "get_device_error", "set_profile_events", "launches_per_call", "exported_symbols",
            "mask_to_seqlens", "gather_rows", "scatter_rows", "unpad", "pad", "fold_pair_bias_row",
            "varlen_attn_decode", "varlen_attn_bwd", "set_wait_limit", "set_test_stall",
-           "BIAS_PAIR_KV_HEADS"]
+           "BIAS_PAIR_KV_HEADS", "varlen_attn"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libvarlen_attn.so")
@@ -531,3 +534,75 @@ def varlen_attn_decode(q, cu_seqlens_q, max_seqlen_q: int, k_cache, v_cache, cac
             ptr(out), ptr(lse), _stream_handle(stream))
     _check(status)
     return out, lse
+
+
+def _autograd_function():
+    import torch
+
+    class _VarlenAttn(torch.autograd.Function):
+        """Forward and backward both run through the C ABI; this class only
+        keeps the forward's output and LSE for the backward and reshapes the
+        per-query-head pair-grid gradient to the grid the caller passed."""
+
+        @staticmethod
+        def forward(ctx, q, k, v, bias_per_key, bias_pair, cu_seqlens_q, cu_seqlens_k,
+                    max_seqlen_q, max_seqlen_k, softmax_scale, causal, bias_pair_kv_heads):
+            out, lse = varlen_attn_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                                       max_seqlen_k, softmax_scale=softmax_scale, causal=causal,
+                                       bias_per_key=bias_per_key, bias_pair=bias_pair,
+                                       bias_pair_kv_heads=bias_pair_kv_heads)
+            ctx.save_for_backward(q, k, v, out, lse, bias_per_key, bias_pair, cu_seqlens_q,
+                                  cu_seqlens_k)
+            ctx.args = (max_seqlen_q, max_seqlen_k, softmax_scale, causal, bias_pair_kv_heads)
+            ctx.mark_non_differentiable(lse)
+            return out, lse
+
+        @staticmethod
+        def backward(ctx, dout, _dlse):
+            q, k, v, out, lse, bk, bp, cu_q, cu_k = ctx.saved_tensors
+            max_q, max_k, scale, causal, kv_heads = ctx.args
+            need_bk = bk is not None and ctx.needs_input_grad[3]
+            need_bp = bp is not None and ctx.needs_input_grad[4]
+            dq, dk, dv, dbk, dbp = varlen_attn_bwd(
+                q, k, v, out, lse, dout.contiguous(), cu_q, cu_k, max_q, max_k,
+                softmax_scale=scale, causal=causal, bias_per_key=bk, bias_pair=bp,
+                bias_pair_kv_heads=kv_heads, need_dbias_per_key=need_bk,
+                need_dbias_pair=need_bp)
+            if need_bp:
+                # per query head [B, Hq, max_q, max_k] -> the grid's own heads
+                # (a broadcast or per-K/V-head grid sums the heads that read
+                # it) and rows / columns (zeros outside the sequences)
+                B, Hq, R, C = dbp.shape
+                Hg = bp.shape[1]
+                dbp = dbp.view(B, Hg, Hq // Hg, R, C).sum(dim=2)
+                grad = torch.zeros(bp.shape, dtype=torch.float32, device=bp.device)
+                r, c = min(R, bp.shape[2]), min(C, bp.shape[3])
+                grad[:, :, :r, :c] = dbp[:, :, :r, :c]
+                dbp = grad
+            return (dq, dk, dv, dbk if need_bk else None, dbp if need_bp else None,
+                    None, None, None, None, None, None, None)
+
+    return _VarlenAttn
+
+
+_VARLEN_ATTN_FN = None
+
+
+def varlen_attn(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                softmax_scale: Optional[float] = None, causal: bool = False, bias_per_key=None,
+                bias_pair=None, bias_pair_kv_heads: bool = False):
+    """Differentiable packed attention (bf16): ``(out, lse)`` with gradients
+    for ``q``, ``k``, ``v``, ``bias_per_key`` and ``bias_pair`` (a 4-D
+    ``[batch, 1 | n_heads | n_kv_heads, rows, cols]`` tensor; a head axis of 1
+    broadcasts, ``bias_pair_kv_heads`` reads it per K/V head) through
+    ``varlen_attn_fwd`` and ``varlen_attn_bwd``."""
+    global _VARLEN_ATTN_FN
+    if _VARLEN_ATTN_FN is None:
+        _VARLEN_ATTN_FN = _autograd_function()
+    if bias_pair is not None and bias_pair.dim() != 4:
+        raise ValueError("varlen_attn takes bias_pair as a 4-D [batch, heads, rows, cols] tensor")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(q.shape[-1])
+    return _VARLEN_ATTN_FN.apply(q, k, v, bias_per_key, bias_pair, cu_seqlens_q, cu_seqlens_k,
+                                 int(max_seqlen_q), int(max_seqlen_k), float(softmax_scale),
+                                 bool(causal), bool(bias_pair_kv_heads))
