@@ -202,3 +202,40 @@ def test_test_stall_setting(lib):
     assert lib.varlen_attn_set_test_stall(1) == 0
     assert lib.varlen_attn_set_test_stall(0) == 0
     va.set_test_stall(False)
+
+
+def test_header_compiles_as_c99_and_links(tmp_path):
+    """A plain C program (no C++, no CUDA headers) includes the header, links
+    the library and calls it: the host-side argument checks answer before any
+    device work, so this runs without a GPU."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "use_abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "varlen_attn.h"
+int main(void) {
+  /* a NULL query pointer is rejected on the host */
+  int rc = varlen_attn_fwd(NULL, NULL, NULL, NULL, NULL, 1, 8, 8, 8, 8, 2, 2, 64, 0.125f, 1,
+                           NULL, NULL, 0, 0, 0, 0, NULL, NULL, NULL);
+  if (rc != VARLEN_ATTN_ERR_NULL_POINTER) { printf("fwd rc %d\n", rc); return 1; }
+  if (strlen(varlen_attn_strerror(rc)) == 0) return 2;
+  if (varlen_attn_version() < 100) return 3;
+  printf("ok %s\n", varlen_attn_strerror(rc));
+  return 0;
+}
+''')
+    exe = tmp_path / "use_abi"
+    libdir = os.path.dirname(va.load_library()._name)
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(root, "include"),
+                        str(src), "-L", libdir, "-lvarlen_attn", f"-Wl,-rpath,{libdir}", "-o",
+                        str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert r.stdout.startswith("ok ")
