@@ -428,7 +428,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_combine_kernel(DecodeParam
 constexpr int kDec2Consumers = 4;
 constexpr int kDec2Threads = 32 * (kDec2Consumers + 1);
 constexpr int kDec2Stages = 4;
-constexpr int kDec2MaxRows = 8;
+constexpr int kDec2MaxRows = 16;
 // Block t goes to stage t % kDec2Stages and consumer warp t % kDec2Consumers.
 // A consumer reaches block t only after block t - kDec2Consumers, so with at
 // least as many stages as consumers the stage's previous fill (block

@@ -788,7 +788,7 @@ int varlen_attn_decode(const void* q, const int32_t* cu_seqlens_q, int batch, in
   const int RT = rows_needed <= 4 ? 4 : rows_needed <= 8 ? 8 : rows_needed <= 16 ? 16 : 32;
   int rc = VARLEN_ATTN_OK;
   if (RT <= kDec2MaxRows) {
-    // up to 8 rows per K/V head: TMA ring, warp-owned key blocks
+    // up to 16 rows per K/V head: TMA ring, warp-owned key blocks
     CUtensorMap tk, tv;
     const int cache_rows = batch * cache_len;
     if (!make_tmap(&tk, k_cache, head_dim, n_kv_heads, cache_rows, kDecKeys) ||
@@ -796,10 +796,12 @@ int varlen_attn_decode(const void* q, const int32_t* cu_seqlens_q, int batch, in
       return VARLEN_ATTN_ERR_CUDA;
     if (head_dim == 64)
       rc = RT == 4 ? launch_decode_tma<64, 4>(grid, tk, tv, dp, st)
-                   : launch_decode_tma<64, 8>(grid, tk, tv, dp, st);
+           : RT == 8 ? launch_decode_tma<64, 8>(grid, tk, tv, dp, st)
+                     : launch_decode_tma<64, 16>(grid, tk, tv, dp, st);
     else
       rc = RT == 4 ? launch_decode_tma<128, 4>(grid, tk, tv, dp, st)
-                   : launch_decode_tma<128, 8>(grid, tk, tv, dp, st);
+           : RT == 8 ? launch_decode_tma<128, 8>(grid, tk, tv, dp, st)
+                     : launch_decode_tma<128, 16>(grid, tk, tv, dp, st);
     if (!rc && splits > 1) {
       if (head_dim == 64) decode_combine_kernel<64><<<rows, kDecThreads, 0, st>>>(dp);
       else decode_combine_kernel<128><<<rows, kDecThreads, 0, st>>>(dp);
