@@ -708,15 +708,16 @@ def run_decode(args, world, rank, local):
     dev = torch.device("cuda", local)
     kc = torch.randn(B, S, Hkv, D, generator=g).to(torch.bfloat16).to(dev)
     vc = torch.randn(B, S, Hkv, D, generator=g).to(torch.bfloat16).to(dev)
-    q = torch.randn(B, Hq, D, generator=g).to(torch.bfloat16).to(dev)
-    cu_q = torch.arange(B + 1, dtype=torch.int32, device=dev)
+    QL = max(1, args.decode_qlen)  # new query tokens per sequence (speculative steps: > 1)
+    q = torch.randn(B * QL, Hq, D, generator=g).to(torch.bfloat16).to(dev)
+    cu_q = torch.arange(B + 1, dtype=torch.int32, device=dev) * QL
     cs = lens.to(dev)
     out = torch.empty_like(q)
-    lse = torch.empty(Hq, B, dtype=torch.float32, device=dev)
+    lse = torch.empty(Hq, B * QL, dtype=torch.float32, device=dev)
     nbytes = int(lens.sum()) * Hkv * D * 2 * 2 + 2 * q.numel() * 2 + lse.numel() * 4
 
     def step():
-        va.varlen_attn_decode(q, cu_q, 1, kc, vc, cs, num_splits=args.decode_splits,
+        va.varlen_attn_decode(q, cu_q, QL, kc, vc, cs, num_splits=args.decode_splits,
                               out=out, lse=lse)
 
     for _ in range(max(3, args.warmup)):
@@ -740,7 +741,7 @@ def run_decode(args, world, rank, local):
         "n_gpus": 1, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 cache and queries; cached lengths U[1024, 8192])",
-        "config": {"workload": "kv_cache_decode", "sequences": B, "q_len": 1, "cache_len": S,
+        "config": {"workload": "kv_cache_decode", "sequences": B, "q_len": QL, "cache_len": S,
                    "cached_tokens": int(lens.sum()), "n_heads": Hq, "n_kv_heads": Hkv,
                    "head_dim": D, "num_splits": args.decode_splits or "auto",
                    "l2": "cache 8.6 GB > 126 MB L2; no flush"},
@@ -840,8 +841,11 @@ def main():
                     help="256 MB scrub write between timed steps; each call timed alone")
     ap.add_argument("--decode", action="store_true",
                     help="time a K/V-cache decode step instead of the forward")
+    ap.add_argument("--decode-qlen", type=int, default=1,
+                    help="--decode: new query tokens per sequence in the step")
     ap.add_argument("--decode-splits", type=int, default=0,
-                    help="--decode: key splits per (sequence, K/V head); 0 = automatic")
+                    help="--decode: 0 = automatic (the tensor-core path when the (sequence, "
+                         "K/V head) pairs fill the GPU); S > 0 = S key ranges on the CUDA cores")
     ap.add_argument("--layout", action="store_true",
                     help="time the packed-layout helpers (unpad, pad) instead of the forward")
     ap.add_argument("--backward", action="store_true",

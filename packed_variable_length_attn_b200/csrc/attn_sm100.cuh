@@ -188,6 +188,7 @@ struct Smem {
   __device__ int* abort_flag() const { return reinterpret_cast<int*>(base + KCfg<D>::kMiscOff + 4); }
 };
 
+template <bool kCache>
 __device__ __forceinline__ Item decode_item(int w, const AttnParams& p) {
   Item it;
   const int2 pr = p.ws.list[w / p.n_hg];
@@ -195,11 +196,19 @@ __device__ __forceinline__ Item decode_item(int w, const AttnParams& p) {
   const int i = pr.x, g = pr.y;
   it.valid = 1;
   it.seq = i;
-  const int q0 = p.cu_q[i], k0 = p.cu_k[i];
+  const int q0 = p.cu_q[i];
   it.Lq = p.cu_q[i + 1] - q0;
-  it.Lk = p.cu_k[i + 1] - k0;
+  int k0;
+  if constexpr (kCache) {  // K/V in place in the cache, packed-GQA rows
+    k0 = i * p.cache_len;
+    it.Lk = p.cache_seqlens[i] + (p.cache_extra ? it.Lq : 0);
+    it.kvh = hg;
+  } else {
+    k0 = p.cu_k[i];
+    it.Lk = p.cu_k[i + 1] - k0;
+    it.kvh = p.pairing == kPairHeads ? hg : hg / p.group;
+  }
   it.kv_row0 = k0;
-  it.kvh = p.pairing == kPairHeads ? hg : hg / p.group;
   fill_slots(it, g, hg, p.pairing, p.group, p.causal);
   it.q_row0[0] = q0 + it.q_loc0[0];
   it.q_row0[1] = q0 + it.q_loc0[1];
@@ -210,7 +219,7 @@ __device__ __forceinline__ Item decode_item(int w, const AttnParams& p) {
 // Runs on all 32 lanes of the load warp (uniform control flow); one elected
 // lane fetches work and issues the copies. Per item: Q of each active slot,
 // then K0, V0, K1, V1, ... (the MMA warp's consumption order).
-template <int D>
+template <int D, bool kCache>
 __device__ void load_role(const Smem<D>& sm, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                           const CUtensorMap* tm_v, const AttnParams& p, const Ctl& ctl) {
   using C = KCfg<D>;
@@ -242,7 +251,7 @@ __device__ void load_role(const Smem<D>& sm, const CUtensorMap* tm_q, const CUte
       const int w = atomicAdd(p.ws.counter, 1);
       Item item;
       if (w < count) {
-        item = decode_item(w, p);
+        item = decode_item<kCache>(w, p);
       } else {
         item.valid = 0;
       }
@@ -258,7 +267,8 @@ __device__ void load_role(const Smem<D>& sm, const CUtensorMap* tm_q, const CUte
         ok = __all_sync(FULL, wait_bar(sm.q_empty(s), (q_uses[s] & 1) ^ 1, ctl));
         ++q_uses[s];
         if (ok && ptx::elect_one()) {
-          ptx::mbar_arrive_expect_tx(sm.q_full(s), C::kQTile);
+          // (a packed-GQA box may write fewer than 128 rows)
+          ptx::mbar_arrive_expect_tx(sm.q_full(s), kCache ? C::kChunks * p.q_box_rows * 128 : C::kQTile);
           for (int c = 0; c < C::kChunks; ++c)
             ptx::tma_load_3d(sm.q(s) + c * C::kQChunk, tm_q, sm.q_full(s), c * 64, item.head[s],
                              item.q_row0[s]);
@@ -331,7 +341,11 @@ __device__ __forceinline__ void issue_pv_half(uint32_t o_tmem, uint32_t p_tmem, 
 // Runs on all 32 lanes of the MMA warp (uniform control flow); one elected
 // lane issues the tensor-core instructions and their commits. The slot loops
 // are unrolled so that every per-slot counter stays in a register.
-template <int D>
+// kCache (K/V cache mode): the rows of a sequence's last V tile past its
+// length are zeroed in shared memory before P V reads the tile. Their
+// probabilities are exactly 0, but the cache may hold anything there
+// (unwritten slots, NaN), and 0 * NaN would reach the output.
+template <int D, bool kCache>
 __device__ void mma_role(const Smem<D>& sm, uint32_t tmem, const Ctl& ctl, int test_stall) {
   using C = KCfg<D>;
   const unsigned FULL = 0xffffffffu;
@@ -360,6 +374,7 @@ __device__ void mma_role(const Smem<D>& sm, uint32_t tmem, const Ctl& ctl, int t
     const Item& itm = sm.items()[k];
     const int valid = itm.valid;
     const int nt[2] = {itm.ntile[0], itm.ntile[1]};
+    const int item_lk = itm.Lk;
     __syncwarp();
     if (ptx::elect_one()) ptx::mbar_arrive(sm.item_empty(k));
     if (!valid) break;
@@ -395,6 +410,18 @@ __device__ void mma_role(const Smem<D>& sm, uint32_t tmem, const Ctl& ctl, int t
     for (int j = 0; j < n && ok; ++j) {
       int vst;
       if (!next_kv(vst)) { ok = false; break; }
+      if (kCache && j == n - 1 && item_lk - j * BN < BN) {
+        const int lane = threadIdx.x & 31;
+        const int keep = item_lk - j * BN;  // rows of the tile inside the sequence
+        uint8_t* vt = sm.kv(vst);
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c)
+          for (int e = lane; e < (BN - keep) * 8; e += 32)  // 16-byte units of 128-byte rows
+            *reinterpret_cast<uint4*>(vt + c * C::kKVChunk + (keep + e / 8) * 128 + (e % 8) * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+      }
       const uint64_t vd = stage_desc<D>(dsc.v0, vst);
       int kst = -1;
 #pragma unroll
@@ -466,7 +493,7 @@ __device__ __forceinline__ void rescale_o(uint32_t t_o, float fac) {
 
 // ------------------------------------------------------------------ softmax
 
-template <int D, bool kBiasKey, bool kBiasPair>
+template <int D, bool kBiasKey, bool kBiasPair, bool kCache>
 __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams& p,
                              const Ctl& ctl) {
   using C = KCfg<D>;
@@ -501,7 +528,11 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
     if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(sm.item_empty(k));
     if (!valid) break;
     if (rows == 0) continue;
-    const int q_loc = q_loc0 + r;
+    // packed GQA: tile row r is token r / G of query head head + r % G
+    constexpr bool pack = kCache;
+    const int r_tok = pack ? r / p.group : r;
+    const int r_head = pack ? head + r % p.group : head;
+    const int q_loc = q_loc0 + r_tok;
     const bool row_ok = r < rows;
     const int limit = p.causal ? min(Lk, q_loc + (Lk - Lq) + 1) : Lk;
     float m_used = -INFINITY, l = 0.f;
@@ -758,8 +789,10 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
         const int x = 8 * k8 + (lane >> 2), cu = lane & 3;
         const uint4 val = ptx::ld_shared_v4(unit_addr(x, cu));
         if (wrow0 + x < rows) {
+          const int xr = wrow0 + x;
+          const int tok = pack ? xr / p.group : xr, hh = pack ? head + xr % p.group : head;
           __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) +
-                               ((long long)(q_row0 + wrow0 + x) * p.n_heads + head) * D + c * 32 + cu * 8;
+                               ((long long)(q_row0 + tok) * p.n_heads + hh) * D + c * 32 + cu * 8;
           *reinterpret_cast<uint4*>(dst) = val;
         }
       }
@@ -770,14 +803,14 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
     }
     if (row_ok && p.lse != nullptr) {
       const float lse = l > 0.f ? (m_used + __log2f(l)) * kLn2 : -INFINITY;
-      p.lse[(long long)head * p.total_q + q_row0 + r] = lse;
+      p.lse[(long long)r_head * p.total_q + q_row0 + r_tok] = lse;
     }
   }
   if constexpr (kBiasKey || kBiasPair) ptx::cp_async_wait_group<0>();  // copies left by an abort
 }
 
 // ------------------------------------------------------------------ kernel
-template <int D, bool kBiasKey, bool kBiasPair>
+template <int D, bool kBiasKey, bool kBiasPair, bool kCache = false>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -827,13 +860,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp < 8) {
     ptx::setmaxnreg_inc<kSoftmaxRegs>();
-    softmax_role<D, kBiasKey, kBiasPair>(sm, tmem, p, ctl);
+    softmax_role<D, kBiasKey, kBiasPair, kCache>(sm, tmem, p, ctl);
   } else {
     ptx::setmaxnreg_dec<kWorkerRegs>();
     if (warp == kMmaWarp) {
-      mma_role<D>(sm, tmem, ctl, p.test_stall);
+      mma_role<D, kCache>(sm, tmem, ctl, p.test_stall);
     } else if (warp == kLoadWarp) {
-      load_role<D>(sm, &tm_q, &tm_k, &tm_v, p, ctl);
+      load_role<D, kCache>(sm, &tm_q, &tm_k, &tm_v, p, ctl);
     }
   }
   ptx::tc_fence_before();

@@ -20,8 +20,13 @@ constexpr int kErrTimeout = 10;
 //                with the next q-block's first one. Both slots read the same
 //                K/V tiles.
 //  kPairQBlocks: two consecutive q-blocks of one head (no GQA sharing).
+//  kPackGQA:     decode-sized queries (Lq * G <= 128 rows): one item per
+//                (sequence, K/V head) whose single slot holds the rows of all
+//                G query heads of the group, row rho = token (rho / G) of
+//                head (rho % G); slot 1 is unused.
 constexpr int kPairHeads = 0;
 constexpr int kPairQBlocks = 1;
+constexpr int kPackGQA = 3;
 
 // Work list in the library workspace (device memory).
 struct Workspace {
@@ -37,12 +42,25 @@ struct SchedParams {
   const int* cu_k;
   int batch, total_q, total_k, max_q, max_k;
   int causal;
-  int pairing;      // kPairHeads / kPairQBlocks; -1 = validate only
+  int pairing;      // kPairHeads / kPairQBlocks / kPackGQA; -1 = validate only
   int group;        // G = Hq / Hkv
   int n_hg;         // work items per (sequence, group) pair
+  // K/V read in place from a per-sequence cache (cache_seqlens != null):
+  // sequence i's keys are rows i*cache_len .. of the cache, Lk_i =
+  // cache_seqlens[i] (+ Lq_i when its new rows were appended); cu_k unused.
+  const int* cache_seqlens;
+  int cache_len, cache_extra;
   Workspace ws;
   int* error;       // device error word
 };
+
+// Key count of sequence i: from cu_seqlens_k, or from the cache lengths.
+template <typename P>
+__device__ __forceinline__ int seq_lk(const P& p, int i) {
+  if (p.cache_seqlens != nullptr)
+    return p.cache_seqlens[i] + (p.cache_extra ? p.cu_q[i + 1] - p.cu_q[i] : 0);
+  return p.cu_k[i + 1] - p.cu_k[i];
+}
 
 struct AttnParams {
   const int* cu_q;
@@ -66,6 +84,10 @@ struct AttnParams {
   long long wait_limit;            // cycles a bounded wait may take
   int test_stall;                  // test hook: the MMA warp first waits on a barrier
                                    // phase nothing completes (its wait runs out)
+  // K/V cache mode (see SchedParams) and the packed-GQA rows of kPackGQA
+  const int* cache_seqlens;
+  int cache_len, cache_extra;
+  int q_box_rows;                  // rows one Q tile load writes (128, or G * (128 / G))
 };
 
 // One CTA work item: up to two 128-row query tiles (slots) that stream the
@@ -103,6 +125,7 @@ __host__ __device__ __forceinline__ int slot_tiles(int q_loc0, int rows, int Lq,
 // its (q-block, head) units per K/V head, or q-block pairs.
 __host__ __device__ __forceinline__ int seq_groups(int Lq, int pairing, int group) {
   const int nqb = ceil_div(Lq, BM);
+  if (pairing == kPackGQA) return 1;
   return pairing == kPairHeads ? ceil_div(group * nqb, 2) : ceil_div(nqb, 2);
 }
 
@@ -110,7 +133,10 @@ __host__ __device__ __forceinline__ int seq_groups(int Lq, int pairing, int grou
 // (local to the K/V group for kPairHeads).
 __host__ __device__ __forceinline__ void slot_unit(int g, int s, int pairing, int group,
                                                    int& q_loc0, int& hl) {
-  if (pairing == kPairHeads) {
+  if (pairing == kPackGQA) {
+    q_loc0 = s == 0 ? 0 : (1 << 29);
+    hl = 0;
+  } else if (pairing == kPairHeads) {
     const int unit = 2 * g + s;
     q_loc0 = (unit / group) * BM;
     hl = unit % group;
@@ -125,11 +151,11 @@ __device__ __forceinline__ void fill_slots(Item& it, int g, int hg, int pairing,
 #pragma unroll
   for (int s = 0; s < 2; ++s) {
     int active, head, q_loc0;
-    if (pairing == kPairHeads) {
+    if (pairing == kPairHeads || pairing == kPackGQA) {
       int hl;
       slot_unit(g, s, pairing, group, q_loc0, hl);
       active = q_loc0 < it.Lq;
-      head = it.kvh * group + hl;
+      head = it.kvh * group + hl;  // kPackGQA: the group's first head
     } else {
       head = hg;
       q_loc0 = (2 * g + s) * BM;
@@ -142,6 +168,7 @@ __device__ __forceinline__ void fill_slots(Item& it, int g, int hg, int pairing,
     it.q_loc0[s] = q_loc0;
     it.rows[s] = rows;
     it.ntile[s] = slot_tiles(q_loc0, rows, it.Lq, it.Lk, causal);
+    if (pairing == kPackGQA) it.rows[s] = rows * group;  // tile rows: tokens x heads
   }
 }
 

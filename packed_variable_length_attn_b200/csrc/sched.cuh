@@ -65,7 +65,7 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int* warp_sums, int* 
 // Sort key of sequence i: size (q-blocks x K/V blocks) descending in the
 // high bits, the index (ascending) in the low 32 bits; keys are unique.
 __device__ __forceinline__ unsigned long long seq_key(const SchedParams& p, int i) {
-  const int lq = p.cu_q[i + 1] - p.cu_q[i], lk = p.cu_k[i + 1] - p.cu_k[i];
+  const int lq = p.cu_q[i + 1] - p.cu_q[i], lk = seq_lk(p, i);
   long long sk = (long long)ceil_div(lq, BM) * ceil_div(lk, BN);
   sk = sk > 0xFFFFFF ? 0xFFFFFF : sk;
   return ((unsigned long long)(0xFFFFFF - sk) << 32) | (unsigned)i;
@@ -132,11 +132,15 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedParams 
   // 1. validation
   int bad = 0;
   for (int i = tid; i <= p.batch; i += kSchedThreads) {
-    const int cq = p.cu_q[i], ck = p.cu_k[i];
+    const int cq = p.cu_q[i];
+    const bool cache = p.cache_seqlens != nullptr;
+    const int ck = cache ? 0 : p.cu_k[i];
     if (i == 0 && (cq != 0 || ck != 0)) bad = 1;
     if (i < p.batch) {
-      const int lq = p.cu_q[i + 1] - cq, lk = p.cu_k[i + 1] - ck;
-      if (lq < 0 || lk < 0 || lq > p.max_q || lk > p.max_k) bad = 1;
+      const int lq = p.cu_q[i + 1] - cq;
+      const int lk = cache ? seq_lk(p, i) : p.cu_k[i + 1] - ck;
+      if (lq < 0 || lk < 0 || lq > p.max_q || lk > (cache ? p.cache_len : p.max_k)) bad = 1;
+      if (cache && p.cache_seqlens[i] < 0) bad = 1;
     } else if (cq > p.total_q || ck > p.total_k) {
       bad = 1;
     }
@@ -250,12 +254,12 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedParams 
   for (int r = warp; r < B; r += kSchedThreads / 32) {
     const int2 o = ord[r];
     const int i = o.x;
-    const int Lq = p.cu_q[i + 1] - p.cu_q[i], Lk = p.cu_k[i + 1] - p.cu_k[i];
+    const int Lq = p.cu_q[i + 1] - p.cu_q[i], Lk = seq_lk(p, i);
     const int ng = seq_groups(Lq, p.pairing, p.group);
     // a pair whose second unit does not exist (the last pair of an odd
     // number of units) may do less work than the pairs before it
     const int units = p.pairing == kPairHeads ? p.group * ceil_div(Lq, BM) : ceil_div(Lq, BM);
-    const bool lone = units & 1;
+    const bool lone = p.pairing != kPackGQA && (units & 1);
     const int m = lone ? ng - 1 : ng;  // full pairs: work non-decreasing in g
     int cnt = m;                         // place of the lone pair
     if (lone) {

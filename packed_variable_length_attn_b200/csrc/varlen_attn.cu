@@ -159,6 +159,22 @@ bool make_tmap(CUtensorMap* m, const void* base, int D, int heads, int rows, int
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map with a box of box_heads heads x box_rows rows (64 columns).
+bool make_tmap_box(CUtensorMap* m, const void* base, int D, int heads, int rows, int box_heads,
+                   int box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)(rows > 0 ? rows : 1)};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) snprintf(t_detail, sizeof t_detail, "cuTensorMapEncodeTiled: CUresult %d", (int)r);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 // Base of a K or V tensor map. With no keys at all (total_k == 0, k and v
@@ -209,10 +225,10 @@ int check_launch(const char* what) {
   return e == cudaSuccess ? VARLEN_ATTN_OK : cuda_fail(what, e);
 }
 
-template <int D, bool BK, bool BP>
+template <int D, bool BK, bool BP, bool CACHE = false>
 int launch_attn(int grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                 const AttnParams& prm, cudaStream_t st) {
-  auto kern = attn_fwd_sm100<D, BK, BP>;
+  auto kern = attn_fwd_sm100<D, BK, BP, CACHE>;
   static thread_local int configured_for = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -349,6 +365,7 @@ int fwd_bf16(const void* q, const void* k, const void* v, const int32_t* cu_seql
     return VARLEN_ATTN_ERR_CUDA;
 
   SchedParams sp;
+  std::memset(&sp, 0, sizeof sp);  // no K/V cache
   sp.cu_q = cu_seqlens_q;
   sp.cu_k = cu_seqlens_k;
   sp.batch = batch;
@@ -365,6 +382,8 @@ int fwd_bf16(const void* q, const void* k, const void* v, const int32_t* cu_seql
   if ((rc = launch_schedule(sp, st))) return rc;
 
   AttnParams prm;
+  std::memset(&prm, 0, sizeof prm);  // no K/V cache
+  prm.q_box_rows = BM;
   prm.cu_q = cu_seqlens_q;
   prm.cu_k = cu_seqlens_k;
   prm.total_q = total_q;
@@ -785,6 +804,71 @@ int varlen_attn_decode(const void* q, const int32_t* cu_seqlens_q, int batch, in
     if (int rc = check_launch("launch decode_append_kernel")) return rc;
   }
   const int rows_needed = max_seqlen_q * G;
+  if (num_splits == 0 && (int64_t)batch * n_kv_heads >= di->sm_count) {
+    // Enough (sequence, K/V head) pairs to fill the GPU: on the tensor cores,
+    // through the packed forward kernel with the K/V read in place from the
+    // cache and the rows of all G query heads of a K/V group in one tile
+    // (token-major: row = token * G + head in group), one work item per
+    // pair, longest first. (With several query rows per K/V head the CUDA-core
+    // kernels below are bound by their fp32 multiply-adds; with one, both are
+    // bound by HBM.) Fewer pairs, or an explicit num_splits: key ranges on
+    // the CUDA cores, merged by LSE.
+    const int box_tok = BM / G;  // tokens of one Q tile load
+    CUtensorMap tq, tk, tv;
+    if (!make_tmap_box(&tq, q, head_dim, n_heads, total_q, G, box_tok) ||
+        !make_tmap(&tk, k_cache, head_dim, n_kv_heads, batch * cache_len, BN) ||
+        !make_tmap(&tv, v_cache, head_dim, n_kv_heads, batch * cache_len, BN))
+      return VARLEN_ATTN_ERR_CUDA;
+    void* wsp = nullptr;
+    if (int rc = workspace(stream, 256 + 2 * (size_t)batch * sizeof(int2), &wsp)) return rc;
+    Workspace ws = carve(wsp, batch);
+    SchedParams sp;
+    std::memset(&sp, 0, sizeof sp);
+    sp.cu_q = cu_seqlens_q;
+    sp.batch = batch;
+    sp.total_q = total_q;
+    sp.total_k = batch * cache_len;
+    sp.max_q = max_seqlen_q;
+    sp.max_k = cache_len;
+    sp.causal = causal ? 1 : 0;
+    sp.pairing = kPackGQA;
+    sp.group = G;
+    sp.n_hg = n_kv_heads;
+    sp.cache_seqlens = cache_seqlens;
+    sp.cache_len = cache_len;
+    sp.cache_extra = k_new != nullptr;
+    sp.ws = ws;
+    sp.error = di->error_word;
+    if (int rc = launch_schedule(sp, st)) return rc;
+    AttnParams prm;
+    std::memset(&prm, 0, sizeof prm);
+    prm.cu_q = cu_seqlens_q;
+    prm.total_q = total_q;
+    prm.n_heads = n_heads;
+    prm.n_kv_heads = n_kv_heads;
+    prm.group = G;
+    prm.pairing = kPackGQA;
+    prm.n_hg = n_kv_heads;
+    prm.causal = causal ? 1 : 0;
+    prm.scale_log2 = softmax_scale * 1.4426950408889634f;
+    prm.scale = softmax_scale;
+    prm.bias_head_div = 1;
+    prm.out = out;
+    prm.lse = lse;
+    prm.ws = ws;
+    prm.error = di->error_word;
+    prm.wait_limit = wait_limit();
+    prm.test_stall = g_test_stall.load(std::memory_order_relaxed);
+    prm.cache_seqlens = cache_seqlens;
+    prm.cache_len = cache_len;
+    prm.cache_extra = k_new != nullptr;
+    prm.q_box_rows = G * box_tok;
+    const int64_t items = (int64_t)batch * n_kv_heads;
+    const int grid = (int)(items < di->sm_count ? items : di->sm_count);
+    int rc = head_dim == 64 ? launch_attn<64, false, false, true>(grid, tq, tk, tv, prm, st)
+                            : launch_attn<128, false, false, true>(grid, tq, tk, tv, prm, st);
+    return rc;
+  }
   const int RT = rows_needed <= 4 ? 4 : rows_needed <= 8 ? 8 : rows_needed <= 16 ? 16 : 32;
   int rc = VARLEN_ATTN_OK;
   if (RT <= kDec2MaxRows) {
@@ -885,6 +969,7 @@ int varlen_attn_bwd(const void* q, const void* k, const void* v, const void* out
   float* delta = reinterpret_cast<float*>(static_cast<char*>(wsp) + 256 + 2 * sizeof(int2));
 
   SchedParams sp;
+  std::memset(&sp, 0, sizeof sp);  // no K/V cache
   sp.cu_q = cu_seqlens_q;
   sp.cu_k = cu_seqlens_k;
   sp.batch = batch;

@@ -134,3 +134,49 @@ def test_decode_cache_overflow_reported():
     va.varlen_attn_decode(q, cu_q, 2, kc, vc, cs, kn, kn.clone())
     assert va.get_device_error() == va.ERR_BAD_SEQLENS
     assert torch.equal(kc[0, :7].cpu(), torch.zeros(7, 1, 64, dtype=torch.bfloat16))
+
+
+# Enough (sequence, K/V head) pairs to fill the GPU: the automatic path runs
+# on the tensor cores (packed forward kernel, K/V read in place from the cache,
+# the G query heads of a group in one tile).
+TC_CASES = [
+    # B, hkv, G, d, q_len, new rows
+    (40, 4, 4, 128, 1, False),
+    (40, 4, 4, 128, 4, True),
+    (160, 1, 7, 64, 2, False),
+    (24, 8, 8, 64, 3, True),
+    (75, 2, 1, 128, 1, True),
+]
+
+
+@pytest.mark.parametrize("case", TC_CASES, ids=lambda c: f"B{c[0]}_kv{c[1]}_G{c[2]}_D{c[3]}_q{c[4]}"
+                         f"{'_new' if c[5] else ''}")
+def test_decode_tensor_core_path_parity(case):
+    B, hkv, G, d, ql, new = case
+    assert B * hkv >= torch.cuda.get_device_properties(0).multi_processor_count
+    hq = hkv * G
+    r = np.random.default_rng(B * 7 + d)
+    cache_len = 2048
+    lq = [ql] * B
+    cl = [int(x) for x in r.integers(0, cache_len - (ql if new else 0) + 1, B)]
+    cl[0] = 0
+    cl[1] = cache_len - (ql if new else 0)
+    cu_q, q, kc, vc, cs, kn, vn = _case(B + d, lq, cl, cache_len, hq, hkv, d, new)
+    # unwritten cache slots past each length hold NaN
+    kcn, vcn = kc.clone(), vc.clone()
+    for i, L in enumerate(cl):
+        kcn[i, L:] = float("nan")
+        vcn[i, L:] = float("nan")
+    kcd, vcd = kcn.cuda(), vcn.cuda()
+    scale = 1.0 / np.sqrt(d)
+    out, lse = va.varlen_attn_decode(q.cuda(), cu_q.cuda(), ql, kcd, vcd, cs.cuda(),
+                                     None if kn is None else kn.cuda(),
+                                     None if vn is None else vn.cuda(), softmax_scale=scale,
+                                     causal=True)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    exp_k = _expected_cache(kc, cs, cu_q, kn)
+    exp_v = _expected_cache(vc, cs, cu_q, vn)
+    lk = [cl[i] + (ql if new else 0) for i in range(B)]
+    ref_o, ref_l = _oracle(q, cu_q, exp_k, exp_v, lk, hq, hkv, scale, True)
+    compare(out, lse, ref_o, ref_l)
