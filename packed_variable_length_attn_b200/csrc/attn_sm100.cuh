@@ -20,6 +20,10 @@
 // P_s (bf16, written back over S_s), and the tensor core accumulates
 // O_s += P_s V_j with P read straight from tensor memory.
 //
+// A cache-mode instantiation (kCache) serves decode steps: K/V tiles are
+// read in place from a per-sequence cache (rows i * cache_len ..), and one
+// slot holds the rows of all G query heads of a K/V group, token-major.
+//
 // Tensor memory (512 columns): S0/P0 [0,128), S1/P1 [128,256),
 // O0 [256, 256+D), O1 [256+D, 256+2D). The softmax publishes P in two halves
 // (keys 0-63, then 64-127), so the first half of P V runs on the tensor core
