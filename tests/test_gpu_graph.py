@@ -86,8 +86,9 @@ def test_forward_replay_bit_identical(config, noalloc):
     assert va.get_device_error() == 0
 
 
-def test_decode_replay_bit_identical():
-    B, Hq, Hkv, D, S = 16, 32, 8, 128, 2048
+@pytest.mark.parametrize("B,Hkv", [(16, 8), (40, 4)])  # CUDA-core path; tensor-core path
+def test_decode_replay_bit_identical(B, Hkv):
+    Hq, D, S = 32, 128, 2048
     gen = torch.Generator().manual_seed(31)
     lens = torch.randint(1, S, (B,), generator=gen, dtype=torch.int32).cuda()
     q = torch.randn(B, Hq, D, generator=gen).to(torch.bfloat16).cuda()
