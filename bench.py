@@ -693,15 +693,17 @@ def run_decode(args, world, rank, local):
     lengths U[1024, 8192] in a [64, 8192, 8, 128] bf16 cache (32/8 heads, the
     long workload's head split). HBM-bound: reported as GB/s of the bytes a
     step must move (cached K and V of every sequence once, q, out, LSE)
-    against the measured HBM peak."""
+    against the measured HBM peak. --sequences B keeps the first B sequences,
+    --decode-cache-len S gives a [B, S, 8, 128] cache with lengths U[S/8, S],
+    --decode-qlen the new tokens per sequence."""
     import torch
     import packed_variable_length_attn_b200 as va
     if rank != 0:
         return
     torch.cuda.set_device(local)
     g = torch.Generator("cpu").manual_seed(20261299)
-    B, S, Hq, Hkv, D = 64, 8192, 32, 8, 128
-    lens = torch.randint(1024, 8192 + 1, (B,), generator=g).to(torch.int32)
+    B, S, Hq, Hkv, D = 64, args.decode_cache_len, 32, 8, 128
+    lens = torch.randint(S // 8, S + 1, (B,), generator=g).to(torch.int32)
     if args.sequences and args.sequences < B:  # small case for profiling
         B = args.sequences
         lens = lens[:B]
@@ -740,11 +742,13 @@ def run_decode(args, world, rank, local):
         "metric": "kv-cache decode step GB/s on 1 B200", "value": gbs, "unit": "GB/s",
         "n_gpus": 1, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) bf16 cache and queries; cached lengths U[1024, 8192])",
+        "data": f"synthetic (seeded N(0,1) bf16 cache and queries; cached lengths "
+                f"U[{S // 8}, {S}])",
         "config": {"workload": "kv_cache_decode", "sequences": B, "q_len": QL, "cache_len": S,
                    "cached_tokens": int(lens.sum()), "n_heads": Hq, "n_kv_heads": Hkv,
                    "head_dim": D, "num_splits": args.decode_splits or "auto",
-                   "l2": "cache 8.6 GB > 126 MB L2; no flush"},
+                   "l2": f"cached K/V read per step {nbytes / 1e6:.0f} MB vs 126 MB L2; "
+                         f"no flush"},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]),
                      "unit": "GB/s", "frac": gbs / float(peaks["hbm_gbs"]),
                      "algorithmic_bytes_per_step": nbytes, "traffic": None,
@@ -844,8 +848,11 @@ def main():
     ap.add_argument("--decode-qlen", type=int, default=1,
                     help="--decode: new query tokens per sequence in the step")
     ap.add_argument("--decode-splits", type=int, default=0,
-                    help="--decode: 0 = automatic (the tensor-core path when the (sequence, "
-                         "K/V head) pairs fill the GPU); S > 0 = S key ranges on the CUDA cores")
+                    help="--decode: 0 = automatic (tensor cores; key ranges of the cache "
+                         "when the (sequence, K/V head) pairs are fewer than the SMs); "
+                         "S > 0 = S key ranges on the CUDA cores")
+    ap.add_argument("--decode-cache-len", type=int, default=8192,
+                    help="--decode: cache rows per sequence S (cached lengths U[S/8, S])")
     ap.add_argument("--layout", action="store_true",
                     help="time the packed-layout helpers (unpad, pad) instead of the forward")
     ap.add_argument("--backward", action="store_true",

@@ -277,21 +277,26 @@ int varlen_attn_bwd(const void* q, const void* k, const void* v, const void* out
  *   max_seqlen_q * (n_heads / n_kv_heads) <= 32 (decode-sized queries; longer
  *   ones belong to varlen_attn_fwd): else VARLEN_ATTN_ERR_BAD_SHAPE.
  *   out [total_q, n_heads, head_dim] bf16, lse [n_heads, total_q] fp32 or NULL.
- *   num_splits: 0 = automatic. When batch * n_kv_heads is at least the
- *            device's SM count the step runs on the tensor cores, one work item
- *            per (sequence, K/V head) with the rows of all G query heads of the
- *            group in one tile (no key ranges). Otherwise, or with num_splits
- *            > 0, it runs on the CUDA cores with the cache's key positions cut
- *            into num_splits equal ranges (whole 32-key blocks; ranges past a
- *            sequence's length are empty and cost one short CTA; automatic:
- *            ranges of at most 1536 keys), one CTA per (range, K/V head,
- *            sequence), partial results in the library workspace merged by a
- *            further launch. Results depend on the path and the ranges in the
- *            last bits (the order of the sums), so give a fixed num_splits where
- *            bitwise reproducibility across batch compositions matters.
- * HBM-bound (every cached key and value is read once): fp32 on the CUDA
- * cores, no bias. Errors as for varlen_attn_fwd; a cache position beyond
- * cache_len raises VARLEN_ATTN_ERR_BAD_SEQLENS on the device.
+ *   num_splits: 0 = automatic: the step runs on the tensor cores, the rows
+ *            of all G query heads of a K/V group in one tile. When batch *
+ *            n_kv_heads is at least the device's SM count, one work item per
+ *            (sequence, K/V head). With fewer pairs, the cache's key positions
+ *            are cut into fixed ranges (multiples of 128 keys, at least 512,
+ *            sized from cache_len and the pair count for about eight work
+ *            items per SM, at most 64 ranges), one work item per (range,
+ *            pair); each range's output, normalised by its own sum, goes in
+ *            fp32 to the library workspace, and a further launch merges the
+ *            ranges by their LSE. num_splits > 0: the step runs on the CUDA
+ *            cores (fp32) with the key positions cut into num_splits equal
+ *            ranges (whole 32-key blocks), one CTA per (range, K/V head,
+ *            sequence), merged the same way. Ranges past a sequence's length
+ *            are empty and only mark their partial LSE as -inf. Results depend
+ *            on the path and the ranges in the last bits (the order of the
+ *            sums), so give a fixed num_splits where bitwise reproducibility
+ *            across batch compositions matters.
+ * HBM-bound (every cached key and value is read once); no bias. Errors as
+ * for varlen_attn_fwd; a cache position beyond cache_len raises
+ * VARLEN_ATTN_ERR_BAD_SEQLENS on the device.
  */
 int varlen_attn_decode(const void* q, const int32_t* cu_seqlens_q, int batch, int total_q,
                        int max_seqlen_q, void* k_cache, void* v_cache, int cache_len,

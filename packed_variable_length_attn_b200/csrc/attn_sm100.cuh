@@ -197,15 +197,20 @@ __device__ __forceinline__ Item decode_item(int w, const AttnParams& p) {
   Item it;
   const int2 pr = p.ws.list[w / p.n_hg];
   const int hg = w % p.n_hg;
-  const int i = pr.x, g = pr.y;
+  // with key ranges a list entry is sequence * ranges + range
+  const int ranges = kCache && p.cache_ranges > 1 ? p.cache_ranges : 1;
+  const int i = pr.x / ranges, rg = pr.x - i * ranges, g = pr.y;
   it.valid = 1;
-  it.seq = i;
+  it.seq = pr.x;
   const int q0 = p.cu_q[i];
   it.Lq = p.cu_q[i + 1] - q0;
-  int k0;
+  int k0, koff = 0;
   if constexpr (kCache) {  // K/V in place in the cache, packed-GQA rows
-    k0 = i * p.cache_len;
-    it.Lk = p.cache_seqlens[i] + (p.cache_extra ? it.Lq : 0);
+    const int lk = p.cache_seqlens[i] + (p.cache_extra ? it.Lq : 0);
+    const int ks = rg * p.range_keys;  // first key of the range
+    k0 = i * p.cache_len + ks;
+    it.Lk = ranges > 1 ? max(0, min(lk - ks, p.range_keys)) : lk;
+    koff = lk - ks - it.Lk;  // keys of the sequence after the range
     it.kvh = hg;
   } else {
     k0 = p.cu_k[i];
@@ -214,6 +219,13 @@ __device__ __forceinline__ Item decode_item(int w, const AttnParams& p) {
   }
   it.kv_row0 = k0;
   fill_slots(it, g, hg, p.pairing, p.group, p.causal);
+  if (kCache && koff > 0) {
+    // A range with keys after it: query token t sees range key c when
+    // c <= t + (Lk + koff - Lq), so the causal mask (and the tiles visited)
+    // take Lq - koff in place of Lq.
+    it.Lq -= koff;
+    it.ntile[0] = slot_tiles(it.q_loc0[0], it.rows[0] / p.group, it.Lq, it.Lk, p.causal);
+  }
   it.q_row0[0] = q0 + it.q_loc0[0];
   it.q_row0[1] = q0 + it.q_loc0[1];
   return it;
@@ -776,28 +788,42 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
 #pragma unroll
       for (int e = 0; e < D; ++e) o[e] = 0u;
     }
+    // a key range of a decode step: its fp32 output, normalised by its own
+    // sum, to the partial buffer (one row per thread; the rows are few)
+    const bool part = kCache && p.part_o != nullptr;
+    const int rg = part ? seq % p.cache_ranges : 0;
+    if (part && row_ok) {
+      float* dst = p.part_o + (((long long)rg * p.total_q + q_row0 + r_tok) * p.n_heads + r_head) * D;
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t vw[16];
+      for (int c = 0; c < D; c += 4)
+        *reinterpret_cast<float4*>(dst + c) =
+            make_float4(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv,
+                        __uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
+    }
+    if (!part) {
 #pragma unroll
-      for (int e = 0; e < 16; ++e)
-        vw[e] = ptx::pack_bf16x2(__uint_as_float(o[c * 32 + 2 * e]) * inv,
-                                 __uint_as_float(o[c * 32 + 2 * e + 1]) * inv);
-      __syncwarp();  // the previous block's reads are done
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t vw[16];
 #pragma unroll
-      for (int u4 = 0; u4 < 4; ++u4)
-        ptx::st_shared_v4(unit_addr(lane, u4), vw[4 * u4], vw[4 * u4 + 1], vw[4 * u4 + 2], vw[4 * u4 + 3]);
-      __syncwarp();
+        for (int e = 0; e < 16; ++e)
+          vw[e] = ptx::pack_bf16x2(__uint_as_float(o[c * 32 + 2 * e]) * inv,
+                                   __uint_as_float(o[c * 32 + 2 * e + 1]) * inv);
+        __syncwarp();  // the previous block's reads are done
 #pragma unroll
-      for (int k8 = 0; k8 < 4; ++k8) {
-        const int x = 8 * k8 + (lane >> 2), cu = lane & 3;
-        const uint4 val = ptx::ld_shared_v4(unit_addr(x, cu));
-        if (wrow0 + x < rows) {
-          const int xr = wrow0 + x;
-          const int tok = pack ? xr / p.group : xr, hh = pack ? head + xr % p.group : head;
-          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) +
-                               ((long long)(q_row0 + tok) * p.n_heads + hh) * D + c * 32 + cu * 8;
-          *reinterpret_cast<uint4*>(dst) = val;
+        for (int u4 = 0; u4 < 4; ++u4)
+          ptx::st_shared_v4(unit_addr(lane, u4), vw[4 * u4], vw[4 * u4 + 1], vw[4 * u4 + 2], vw[4 * u4 + 3]);
+        __syncwarp();
+#pragma unroll
+        for (int k8 = 0; k8 < 4; ++k8) {
+          const int x = 8 * k8 + (lane >> 2), cu = lane & 3;
+          const uint4 val = ptx::ld_shared_v4(unit_addr(x, cu));
+          if (wrow0 + x < rows) {
+            const int xr = wrow0 + x;
+            const int tok = pack ? xr / p.group : xr, hh = pack ? head + xr % p.group : head;
+            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) +
+                                 ((long long)(q_row0 + tok) * p.n_heads + hh) * D + c * 32 + cu * 8;
+            *reinterpret_cast<uint4*>(dst) = val;
+          }
         }
       }
     }
@@ -805,9 +831,10 @@ __device__ void softmax_role(const Smem<D>& sm, uint32_t tmem, const AttnParams&
       ptx::tc_fence_before();
       ptx::mbar_arrive(sm.o_empty(wg));
     }
-    if (row_ok && p.lse != nullptr) {
+    float* lse_out = part ? p.part_lse + (long long)rg * p.n_heads * p.total_q : p.lse;
+    if (row_ok && lse_out != nullptr) {
       const float lse = l > 0.f ? (m_used + __log2f(l)) * kLn2 : -INFINITY;
-      p.lse[(long long)r_head * p.total_q + q_row0 + r_tok] = lse;
+      lse_out[(long long)r_head * p.total_q + q_row0 + r_tok] = lse;
     }
   }
   if constexpr (kBiasKey || kBiasPair) ptx::cp_async_wait_group<0>();  // copies left by an abort

@@ -50,6 +50,10 @@ struct SchedParams {
   // cache_seqlens[i] (+ Lq_i when its new rows were appended); cu_k unused.
   const int* cache_seqlens;
   int cache_len, cache_extra;
+  // Key ranges (cache mode, cache_ranges > 1): the list is built over
+  // batch * cache_ranges virtual sequences, j = i * cache_ranges + r holding
+  // keys [r * range_keys, (r + 1) * range_keys) of sequence i (range_lk).
+  int cache_ranges, range_keys;
   Workspace ws;
   int* error;       // device error word
 };
@@ -60,6 +64,23 @@ __device__ __forceinline__ int seq_lk(const P& p, int i) {
   if (p.cache_seqlens != nullptr)
     return p.cache_seqlens[i] + (p.cache_extra ? p.cu_q[i + 1] - p.cu_q[i] : 0);
   return p.cu_k[i + 1] - p.cu_k[i];
+}
+
+// Key count of virtual sequence j when the cache's keys are cut into ranges
+// (sequence j / cache_ranges, range j % cache_ranges); seq_lk without ranges.
+template <typename P>
+__device__ __forceinline__ int range_lk(const P& p, int j) {
+  if (p.cache_ranges <= 1) return seq_lk(p, j);
+  const int i = j / p.cache_ranges;
+  const int left = seq_lk(p, i) - (j - i * p.cache_ranges) * p.range_keys;
+  return left < 0 ? 0 : left < p.range_keys ? left : p.range_keys;
+}
+
+// Query rows of virtual sequence j (those of sequence j / cache_ranges).
+template <typename P>
+__device__ __forceinline__ int range_lq(const P& p, int j) {
+  const int i = p.cache_ranges > 1 ? j / p.cache_ranges : j;
+  return p.cu_q[i + 1] - p.cu_q[i];
 }
 
 struct AttnParams {
@@ -88,6 +109,12 @@ struct AttnParams {
   const int* cache_seqlens;
   int cache_len, cache_extra;
   int q_box_rows;                  // rows one Q tile load writes (128, or G * (128 / G))
+  // Key ranges (see SchedParams): each range's output, normalised by its own
+  // sum, goes to part_o [ranges, Tq, Hq, D] fp32 and its LSE to part_lse
+  // [ranges, Hq, Tq]; a split-combine kernel merges them.
+  int cache_ranges, range_keys;
+  float* part_o;
+  float* part_lse;
 };
 
 // One CTA work item: up to two 128-row query tiles (slots) that stream the

@@ -26,6 +26,9 @@
 // instead of being fetched from HBM again for every q-block; largest first
 // within and across sequences keeps the longest items away from the end.
 // The order only decides when an item runs, never what it computes.
+// With key ranges (a decode step whose sequences are cut into ranges of the
+// cache, see SchedParams) steps 2-4 run over the virtual sequences, one per
+// (sequence, range), each sized by its own keys.
 #pragma once
 #include "common.cuh"
 
@@ -65,7 +68,7 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int* warp_sums, int* 
 // Sort key of sequence i: size (q-blocks x K/V blocks) descending in the
 // high bits, the index (ascending) in the low 32 bits; keys are unique.
 __device__ __forceinline__ unsigned long long seq_key(const SchedParams& p, int i) {
-  const int lq = p.cu_q[i + 1] - p.cu_q[i], lk = seq_lk(p, i);
+  const int lq = range_lq(p, i), lk = range_lk(p, i);
   long long sk = (long long)ceil_div(lq, BM) * ceil_div(lk, BN);
   sk = sk > 0xFFFFFF ? 0xFFFFFF : sk;
   return ((unsigned long long)(0xFFFFFF - sk) << 32) | (unsigned)i;
@@ -165,7 +168,7 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedParams 
 
   // 2. sequences by size. `ord` ends up holding, per rank, the sequence index
   // (x) and, after step 3, the first list position of its pairs (y).
-  const int B = p.batch;
+  const int B = p.batch * (p.cache_ranges > 1 ? p.cache_ranges : 1);
   int2* ord;
   if (B <= kSeqSortCap) {
     int n = 1;
@@ -231,7 +234,7 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedParams 
     int ng = 0, i = 0;
     if (r < B) {
       i = ord[r].x;
-      ng = seq_groups(p.cu_q[i + 1] - p.cu_q[i], p.pairing, p.group);
+      ng = seq_groups(range_lq(p, i), p.pairing, p.group);
     }
     const int off = carry + block_exclusive_scan(ng, s_warp, &s_total);
     if (r < B) ord[r].y = off;
@@ -254,7 +257,7 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedParams 
   for (int r = warp; r < B; r += kSchedThreads / 32) {
     const int2 o = ord[r];
     const int i = o.x;
-    const int Lq = p.cu_q[i + 1] - p.cu_q[i], Lk = seq_lk(p, i);
+    const int Lq = range_lq(p, i), Lk = range_lk(p, i);
     const int ng = seq_groups(Lq, p.pairing, p.group);
     // a pair whose second unit does not exist (the last pair of an odd
     // number of units) may do less work than the pairs before it

@@ -46,6 +46,13 @@ __device__ int g_device_error = 0;
 
 constexpr int kVersion = 100;  // 0.1.0
 
+// Key ranges of the tensor-core decode path (used when the (sequence, K/V
+// head) pairs are fewer than the SMs): about this many work items per SM were
+// every sequence full, ranges of at least this many keys, at most this many.
+constexpr int kRangeItemsPerSm = 8;
+constexpr int kMinRangeKeys = 512;
+constexpr int kMaxRanges = 64;
+
 struct DeviceInfo {
   bool init = false;
   int sm_count = 0;
@@ -784,14 +791,6 @@ int varlen_attn_decode(const void* q, const int32_t* cu_seqlens_q, int batch, in
   dp.part_o = nullptr;
   dp.part_lse = nullptr;
   dp.error = di->error_word;
-  if (splits > 1) {
-    const size_t po = (size_t)splits * total_q * n_heads * head_dim * sizeof(float);
-    const size_t pl = (size_t)splits * n_heads * total_q * sizeof(float);
-    void* wsp = nullptr;
-    if (int rc = workspace(stream, po + pl, &wsp)) return rc;
-    dp.part_o = static_cast<float*>(wsp);
-    dp.part_lse = reinterpret_cast<float*>(static_cast<char*>(wsp) + po);
-  }
   const dim3 grid(splits, n_kv_heads, batch);
   const int rows = (int)std::min<int64_t>((int64_t)total_q * n_heads / (kDecThreads / 32) + 1,
                                           (int64_t)di->sm_count * 16);
@@ -804,15 +803,36 @@ int varlen_attn_decode(const void* q, const int32_t* cu_seqlens_q, int batch, in
     if (int rc = check_launch("launch decode_append_kernel")) return rc;
   }
   const int rows_needed = max_seqlen_q * G;
-  if (num_splits == 0 && (int64_t)batch * n_kv_heads >= di->sm_count) {
-    // Enough (sequence, K/V head) pairs to fill the GPU: on the tensor cores,
-    // through the packed forward kernel with the K/V read in place from the
-    // cache and the rows of all G query heads of a K/V group in one tile
-    // (token-major: row = token * G + head in group), one work item per
-    // pair, longest first. (With several query rows per K/V head the CUDA-core
-    // kernels below are bound by their fp32 multiply-adds; with one, both are
-    // bound by HBM.) Fewer pairs, or an explicit num_splits: key ranges on
-    // the CUDA cores, merged by LSE.
+  if (num_splits == 0) {
+    // On the tensor cores, through the packed forward kernel with the K/V
+    // read in place from the cache and the rows of all G query heads of a
+    // K/V group in one tile (token-major: row = token * G + head in group),
+    // longest first. (With several query rows per K/V head the CUDA-core
+    // kernels below are bound by their fp32 multiply-adds; with one, both
+    // are bound by HBM.) With enough (sequence, K/V head) pairs to fill the
+    // GPU, one work item per pair; with fewer, each sequence's keys are cut
+    // into fixed ranges of the cache, one work item per (range, pair), whose
+    // outputs the split-combine kernel merges by LSE. The ranges are sized
+    // for about kRangeItemsPerSm items per SM were every sequence at
+    // cache_len (the lengths are on the device), and hold at least
+    // kMinRangeKeys keys.
+    const int64_t pairs = (int64_t)batch * n_kv_heads;
+    int ranges = 1, range_keys = 0;
+    if (pairs < di->sm_count) {
+      const int64_t want = (kRangeItemsPerSm * (int64_t)di->sm_count + pairs - 1) / pairs;
+      const int most = std::max(1, cache_len / kMinRangeKeys);
+      ranges = (int)std::min<int64_t>(want, std::min(most, kMaxRanges));
+      range_keys = ceil_div(ceil_div(cache_len, ranges), BN) * BN;
+      ranges = ceil_div(cache_len, range_keys);  // no range starts past the cache
+      if (ranges <= 1) {
+        ranges = 1;
+        range_keys = 0;
+      }
+    }
+    const int cap = batch * ranges;  // list entries: (sequence, range) pairs
+    const size_t list_bytes = (256 + 2 * (size_t)cap * sizeof(int2) + 255) / 256 * 256;
+    const size_t po = ranges > 1 ? (size_t)ranges * total_q * n_heads * head_dim * sizeof(float) : 0;
+    const size_t pl = ranges > 1 ? (size_t)ranges * n_heads * total_q * sizeof(float) : 0;
     const int box_tok = BM / G;  // tokens of one Q tile load
     CUtensorMap tq, tk, tv;
     if (!make_tmap_box(&tq, q, head_dim, n_heads, total_q, G, box_tok) ||
@@ -820,8 +840,10 @@ int varlen_attn_decode(const void* q, const int32_t* cu_seqlens_q, int batch, in
         !make_tmap(&tv, v_cache, head_dim, n_kv_heads, batch * cache_len, BN))
       return VARLEN_ATTN_ERR_CUDA;
     void* wsp = nullptr;
-    if (int rc = workspace(stream, 256 + 2 * (size_t)batch * sizeof(int2), &wsp)) return rc;
-    Workspace ws = carve(wsp, batch);
+    if (int rc = workspace(stream, list_bytes + po + pl, &wsp)) return rc;
+    Workspace ws = carve(wsp, cap);
+    float* part_o = ranges > 1 ? reinterpret_cast<float*>(static_cast<char*>(wsp) + list_bytes) : nullptr;
+    float* part_lse = ranges > 1 ? reinterpret_cast<float*>(static_cast<char*>(wsp) + list_bytes + po) : nullptr;
     SchedParams sp;
     std::memset(&sp, 0, sizeof sp);
     sp.cu_q = cu_seqlens_q;
@@ -837,6 +859,8 @@ int varlen_attn_decode(const void* q, const int32_t* cu_seqlens_q, int batch, in
     sp.cache_seqlens = cache_seqlens;
     sp.cache_len = cache_len;
     sp.cache_extra = k_new != nullptr;
+    sp.cache_ranges = ranges;
+    sp.range_keys = range_keys;
     sp.ws = ws;
     sp.error = di->error_word;
     if (int rc = launch_schedule(sp, st)) return rc;
@@ -863,11 +887,31 @@ int varlen_attn_decode(const void* q, const int32_t* cu_seqlens_q, int batch, in
     prm.cache_len = cache_len;
     prm.cache_extra = k_new != nullptr;
     prm.q_box_rows = G * box_tok;
-    const int64_t items = (int64_t)batch * n_kv_heads;
+    prm.cache_ranges = ranges;
+    prm.range_keys = range_keys;
+    prm.part_o = part_o;
+    prm.part_lse = part_lse;
+    const int64_t items = pairs * ranges;
     const int grid = (int)(items < di->sm_count ? items : di->sm_count);
     int rc = head_dim == 64 ? launch_attn<64, false, false, true>(grid, tq, tk, tv, prm, st)
                             : launch_attn<128, false, false, true>(grid, tq, tk, tv, prm, st);
+    if (!rc && ranges > 1) {
+      dp.n_splits = ranges;
+      dp.part_o = part_o;
+      dp.part_lse = part_lse;
+      if (head_dim == 64) decode_combine_kernel<64><<<rows, kDecThreads, 0, st>>>(dp);
+      else decode_combine_kernel<128><<<rows, kDecThreads, 0, st>>>(dp);
+      rc = check_launch("launch decode_combine_kernel");
+    }
     return rc;
+  }
+  if (splits > 1) {
+    const size_t po = (size_t)splits * total_q * n_heads * head_dim * sizeof(float);
+    const size_t pl = (size_t)splits * n_heads * total_q * sizeof(float);
+    void* wsp = nullptr;
+    if (int rc = workspace(stream, po + pl, &wsp)) return rc;
+    dp.part_o = static_cast<float*>(wsp);
+    dp.part_lse = reinterpret_cast<float*>(static_cast<char*>(wsp) + po);
   }
   const int RT = rows_needed <= 4 ? 4 : rows_needed <= 8 ? 8 : rows_needed <= 16 ? 16 : 32;
   int rc = VARLEN_ATTN_OK;

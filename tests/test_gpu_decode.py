@@ -180,3 +180,61 @@ def test_decode_tensor_core_path_parity(case):
     lk = [cl[i] + (ql if new else 0) for i in range(B)]
     ref_o, ref_l = _oracle(q, cu_q, exp_k, exp_v, lk, hq, hkv, scale, True)
     compare(out, lse, ref_o, ref_l)
+
+
+# Fewer (sequence, K/V head) pairs than SMs: the automatic path still runs on
+# the tensor cores, each sequence's keys cut into fixed ranges of the cache
+# (at least 512 keys, a multiple of the 128-key tile), one work item per
+# (range, pair), the ranges' outputs merged by LSE. The lengths sit on and
+# next to multiples of 512 and at both ends, and several new tokens put the
+# causal diagonal across a range boundary (a sequence of 513 keys has a
+# one-key last range, so the earlier tokens see only part of the range before).
+RANGE_CASES = [
+    # B, hkv, G, d, q_len, new rows, cache_len
+    (8, 4, 4, 128, 1, False, 4096),
+    (8, 4, 4, 128, 4, True, 4096),
+    (7, 2, 7, 64, 2, False, 3000),
+    (2, 8, 4, 64, 8, True, 8192),
+    (6, 1, 1, 128, 16, True, 2048),
+    (8, 3, 4, 128, 4, False, 4096),
+]
+
+
+@pytest.mark.parametrize("case", RANGE_CASES, ids=lambda c: f"B{c[0]}_kv{c[1]}_G{c[2]}_D{c[3]}"
+                         f"_q{c[4]}{'_new' if c[5] else ''}_S{c[6]}")
+def test_decode_key_range_path_parity(case):
+    B, hkv, G, d, ql, new, cache_len = case
+    assert B * hkv < torch.cuda.get_device_properties(0).multi_processor_count
+    hq = hkv * G
+    r = np.random.default_rng(B * 11 + d + cache_len)
+    extra = ql if new else 0
+    targets = [0, 1, 512, 513, 1023, 1029, cache_len, 2 * 512 + 3]
+    lk = [max(extra, min(cache_len, t)) for t in targets[:B]]
+    if B > len(targets):
+        lk += [int(x) for x in r.integers(extra, cache_len + 1, B - len(targets))]
+    cl = [L - extra for L in lk]
+    cu_q, q, kc, vc, cs, kn, vn = _case(B * 13 + d, [ql] * B, cl, cache_len, hq, hkv, d, new)
+    kcn, vcn = kc.clone(), vc.clone()  # unwritten cache slots past each length hold NaN
+    for i, L in enumerate(cl):
+        kcn[i, L:] = float("nan")
+        vcn[i, L:] = float("nan")
+    scale = 1.0 / np.sqrt(d)
+    outs = []
+    for _ in range(2):
+        kcd, vcd = kcn.cuda(), vcn.cuda()
+        out, lse = va.varlen_attn_decode(q.cuda(), cu_q.cuda(), ql, kcd, vcd, cs.cuda(),
+                                         None if kn is None else kn.cuda(),
+                                         None if vn is None else vn.cuda(),
+                                         softmax_scale=scale, causal=True)
+        torch.cuda.synchronize()
+        outs.append((out, lse))
+    assert torch.isfinite(outs[0][0].float()).all()
+    for a, b in zip(outs[0], outs[1]):  # deterministic run to run
+        assert torch.equal(a.contiguous().view(torch.int32 if a.dtype == torch.float32
+                                               else torch.int16),
+                           b.contiguous().view(torch.int32 if b.dtype == torch.float32
+                                               else torch.int16))
+    exp_k = _expected_cache(kc, cs, cu_q, kn)
+    exp_v = _expected_cache(vc, cs, cu_q, vn)
+    ref_o, ref_l = _oracle(q, cu_q, exp_k, exp_v, lk, hq, hkv, scale, True)
+    compare(outs[0][0], outs[0][1], ref_o, ref_l)

@@ -86,8 +86,10 @@ def test_forward_replay_bit_identical(config, noalloc):
     assert va.get_device_error() == 0
 
 
-@pytest.mark.parametrize("B,Hkv", [(16, 8), (40, 4)])  # CUDA-core path; tensor-core path
-def test_decode_replay_bit_identical(B, Hkv):
+# tensor cores with key ranges (16 x 8 pairs, fewer than the SMs); tensor
+# cores, one item per pair; the CUDA-core kernel (explicit key ranges)
+@pytest.mark.parametrize("B,Hkv,splits", [(16, 8, 0), (40, 4, 0), (16, 8, 4)])
+def test_decode_replay_bit_identical(B, Hkv, splits):
     Hq, D, S = 32, 128, 2048
     gen = torch.Generator().manual_seed(31)
     lens = torch.randint(1, S, (B,), generator=gen, dtype=torch.int32).cuda()
@@ -99,7 +101,7 @@ def test_decode_replay_bit_identical(B, Hkv):
     lse = torch.empty(Hq, B, device="cuda")
 
     def call(o=out, l=lse):
-        va.varlen_attn_decode(q, cu, 1, kc, vc, lens, out=o, lse=l)
+        va.varlen_attn_decode(q, cu, 1, kc, vc, lens, num_splits=splits, out=o, lse=l)
 
     g = _capture(call)
     for seed in (None, 12):
