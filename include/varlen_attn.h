@@ -259,11 +259,12 @@ int varlen_attn_bwd(const void* q, const void* k, const void* v, const void* out
                     int64_t dbias_stride_q, void* stream);
 
 /*
- * Decode attention over a per-sequence K/V cache (flash_attn_with_kvcache in
- * "fix(flex): avoid decoding kernel selection for short GQA" and the noether
- * attention module page; q_len = 1 decode steps, FDMA integration page,
- * Causality Handling). Same definition as varlen_attn_fwd with the keys and
- * values of sequence i taken from the cache:
+ * Decode attention over a per-sequence K/V cache (flash_attn_with_kvcache,
+ * listed by the noether attention module page, module; the decoding-kernel
+ * path that short GQA rows can reach, "fix(flex): avoid decoding kernel
+ * selection for short GQA", Outcome; q_len = 1 decode steps, FDMA
+ * integration page, Causality Handling). Same definition as varlen_attn_fwd
+ * with the keys and values of sequence i taken from the cache:
  *
  *   k_cache, v_cache  [batch, cache_len, n_kv_heads, head_dim] bf16; sequence
  *            i's cached rows are i*cache_len .. i*cache_len + cache_seqlens[i]-1.
